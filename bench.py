@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward on B200: tokens/s of the whole hot path
+(routing, dispatch, grouped SwiGLU experts, combine, bias step) at the
+DeepSeek-V3 shape, with the roofline fraction of its dominant kernel.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = moe_layer_forward over one fresh batch of T tokens followed by the
+aux-loss-free bias step (the bias is carried from step to step).  Inputs are
+synthetic (moe_inputs) and resident in HBM before the timed region; the expert
+weights (22.6 GB) are far larger than L2, so no flush is needed.  N > 1 runs N
+independent replicas (one process per GPU, no collective in the data path):
+weak scaling, timed as the max over ranks.
+
+--impl reference times the CPU oracle (oracle/) on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s @DeepSeek-V3 shape; % of bf16 tensor/HBM roofline"
+DEFAULT_WORKLOAD = "deepseek_v3"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of the layer and of its kernels
+# ---------------------------------------------------------------------------
+
+def layer_work(w, kept: np.ndarray):
+    """(flops, bytes) of one layer step by the roofline definition: router
+    GEMM + SwiGLU of every kept row and shared row; touched expert weights,
+    shared weights, centroids, h in and y out."""
+    n_rows = int(kept.sum())
+    touched = int((kept > 0).sum())
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    flops = 2 * d * w.E_r * w.T + 6 * d * f * n_rows + 6 * d * fs * w.E_s * w.T
+    es = 2 if w.dtype == "bf16" else 4
+    nbytes = (touched * 3 * d * f * es + w.E_s * 3 * d * fs * es + w.E_r * d * 4
+              + 2 * w.T * d * es)
+    return flops, nbytes
+
+
+def gateup_work(w, kept: np.ndarray):
+    """(flops, bytes) of one launch of the gate/up grouped GEMM: touched gate+up
+    weights, one read of the permuted rows (and of h for the shared experts),
+    one write of the SwiGLU products."""
+    n_rows = int(kept.sum())
+    touched = int((kept > 0).sum())
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    rows_s = w.E_s * w.T
+    flops = 4 * d * (f * n_rows + fs * rows_s)
+    nbytes = 2 * (touched * 2 * d * f + w.E_s * 2 * d * fs + (n_rows + min(rows_s, w.T)) * d
+                  + n_rows * f + rows_s * fs)
+    return flops, nbytes
+
+
+def down_work(w, kept: np.ndarray):
+    n_rows = int(kept.sum())
+    touched = int((kept > 0).sum())
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    rows_s = w.E_s * w.T
+    flops = 2 * d * (f * n_rows + fs * rows_s)
+    nbytes = 2 * (touched * d * f + w.E_s * d * fs + n_rows * f + rows_s * fs + (n_rows + rows_s) * d)
+    return flops, nbytes
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+_WCACHE = __import__("collections").OrderedDict()   # (which, expert) -> host weights
+_WCACHE_MAX = 192
+
+
+def oracle_sample_time(w, tokens: np.ndarray, step: int = 0):
+    """Time the oracle's layer forward (affinity, selection, gates, dispatch,
+    experts, combine) on a sample of tokens of step `step`; the expert weights
+    it needs are generated before the clock starts."""
+    from moe_inputs import native
+    from oracle import moe_oracle as mo
+    h = np.stack([mi.gen_h(w, step, slice(int(t), int(t) + 1))[0] for t in tokens])
+    e = mi.gen_centroids(w)
+    b = mi.gen_bias(w)
+    cfg = mo.LayerConfig(T=len(tokens), d_model=w.d_model, E_r=w.E_r, E_s=w.E_s, K=w.K,
+                         score_fn=w.score_fn, n_groups=w.n_groups, topk_groups=w.topk_groups,
+                         group_topn=w.group_topn, capacity_factor=w.capacity_factor,
+                         add_residual=w.add_residual)
+    s = mo.affinity(h, e, w.score_fn)
+    idx = mo.select_experts(s, b, w.K, w.n_groups, w.topk_groups, w.group_topn)
+    need = [(which, int(ex)) for ex in np.unique(idx) for which in ("gate", "up", "down")]
+    need += [(which, j) for j in range(w.E_s) for which in ("sgate", "sup", "sdown")]
+    for key in need:
+        if key in _WCACHE:
+            _WCACHE.move_to_end(key)
+        else:
+            _WCACHE[key] = native.weight_host(w, *key)
+            while len(_WCACHE) > _WCACHE_MAX:
+                _WCACHE.popitem(last=False)
+    src = lambda which, ex: _WCACHE[(which, int(ex))]
+    t0 = time.perf_counter()
+    mo.layer_forward(cfg, h, e, b, src)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, n_tokens: int):
+    rng = np.random.default_rng(12345)
+    tokens = np.sort(rng.choice(w.T, size=n_tokens, replace=False))
+    dt = oracle_sample_time(w, tokens)
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} of the {w.T} tokens of one batch (seeded sample), full layer "
+                      f"forward on them in float64 numpy; weight generation excluded",
+            "seconds": dt}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    per_step = args.ref_tokens
+    times = []
+    for i in range(args.warmup + args.steps):
+        rng = np.random.default_rng(1000 + i)
+        tokens = np.sort(rng.choice(w.T, size=per_step, replace=False))
+        dt = oracle_sample_time(w, tokens, step=i % max(1, w.steps))
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = per_step * len(times) / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * total / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: {per_step} seeded tokens of the batch, full layer "
+                                       f"forward in float64 numpy"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "T": w.T, "d_model": w.d_model, "E_r": w.E_r, "E_s": w.E_s, "K": w.K,
+            "d_ffn": w.d_ffn, "d_ffn_shared": w.d_ffn_shared,
+            "routing": "sigmoid, bias-only selection" if w.score_fn == 0 else "softmax",
+            "groups": f"{w.n_groups} groups, keep {w.topk_groups}, group score = top-{w.group_topn} sum"
+            if w.n_groups > 1 else "none",
+            "bias_step": f"gamma={w.gamma} every step" if w.gamma else "none",
+            "capacity_factor": w.capacity_factor,
+            "l2": "inputs larger than L2 (expert weights stream from HBM every step)"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_mixture_experts_selection_b200 as moe
+    from moe_inputs import native
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    bf16 = w.dtype == "bf16"
+    dt = torch.bfloat16 if bf16 else torch.float32
+
+    # ---- inputs resident in HBM ----
+    W = {}
+    for k in ("gate", "up", "down", "sgate", "sup", "sdown"):
+        tid, n, rows, cols, sigma = mi.weight_spec(w, k)
+        if n == 0:
+            W[k] = None
+            continue
+        t = torch.empty((n, rows, cols), dtype=dt, device=dev)
+        native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, tid, 0, sigma, stream=stream.cuda_stream)
+        W[k] = t
+    e = torch.from_numpy(mi.gen_centroids(w)).to(dev)
+    b = torch.from_numpy(mi.gen_bias(w)).to(dev)
+    n_steps = args.warmup + args.steps
+    H = []
+    for i in range(n_steps):
+        t = torch.empty((w.T, w.d_model), dtype=dt, device=dev)
+        native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, mi.h_tensor_id(rank * 100000 + i), 0, 1.0,
+                           stream=stream.cuda_stream)
+        H.append(t)
+    cfg = moe.config_for(w)
+    ws = moe.alloc_workspace(moe.moe_workspace_size(cfg), dev)
+    y = torch.empty((w.T, w.d_model), dtype=dt, device=dev)
+    kept = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
+    counts = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
+    max_vio = torch.zeros(n_steps, dtype=torch.float32, device=dev)
+    update = w.gamma > 0
+
+    def step(i, hh=None):
+        moe.moe_layer_forward(cfg, H[i] if hh is None else hh, e, b, W["gate"], W["up"], W["down"],
+                              W["sgate"], W["sup"], W["sdown"], y, ws, counts_out=counts[i],
+                              kept_out=kept[i], update_bias=update, gamma=w.gamma,
+                              max_vio_out=max_vio[i:i + 1])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    b_after_warmup = b.clone()
+
+    # phase events per timed step
+    n_ph = len(moe.PHASES) + 1
+    ph_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ph)] for _ in range(args.steps)]
+    for evs in ph_events:
+        for ev in evs:
+            ev.record()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t_start.record()
+        for j in range(args.steps):
+            moe.moe_set_phase_events(ph_events[j])
+            step(args.warmup + j)
+        t_end.record()
+        torch.cuda.synchronize()
+    moe.moe_set_phase_events([])
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    err = moe.moe_get_device_error(ws)
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed region")
+
+    phase_ms = np.array([[evs[i].elapsed_time(evs[i + 1]) for i in range(n_ph - 1)] for evs in ph_events])
+    kept_h = kept.cpu().numpy()[args.warmup:]
+    vio_h = max_vio.cpu().numpy()
+    value = world * w.T * args.steps / (elapsed_ms / 1000.0)
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        pin_h = [H[i].cpu().pin_memory() for i in range(args.warmup, n_steps)]
+        y_host = torch.empty((w.T, w.d_model), dtype=dt).pin_memory()
+        h_dev = torch.empty_like(H[0])
+        b.copy_(b_after_warmup)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for j in range(args.steps):
+            h_dev.copy_(pin_h[j], non_blocking=True)
+            step(args.warmup + j, h_dev)
+            y_host.copy_(y, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        es = 2 if bf16 else 4
+        e2e = {"value": world * w.T * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": w.T * w.d_model * es, "d2h_bytes_per_step": w.T * w.d_model * es}
+
+    if rank != 0:
+        return
+
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    bf16_peak = float(peaks["bf16_tflops_sustained"])
+    # dominant kernel: the gate/up grouped GEMM
+    gu_ms = phase_ms[:, moe.PHASES.index("ffn_gate_up")]
+    dn_ms = phase_ms[:, moe.PHASES.index("ffn_down")]
+    gu = [gateup_work(w, k) for k in kept_h]
+    dn = [down_work(w, k) for k in kept_h]
+    gu_bytes = float(np.mean([x[1] for x in gu]))
+    gu_flops = float(np.mean([x[0] for x in gu]))
+    gu_s = float(np.mean(gu_ms)) / 1000.0
+    achieved = gu_bytes / gu_s / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get(w.name, {}).get("ffn_gate_up")
+    layer = [layer_work(w, k) for k in kept_h]
+    l_flops = float(np.mean([x[0] for x in layer]))
+    l_bytes = float(np.mean([x[1] for x in layer]))
+    t_roof = max(l_flops / (bf16_peak * 1e12), l_bytes / (hbm * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if bf16 else "f32",
+        "data": "synthetic", "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "kernel": "ffn_gate_up (tcgen05 grouped GEMM)",
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "tensor_tflops": gu_flops / gu_s / 1e12,
+                     "tensor_frac_sustained": gu_flops / gu_s / 1e12 / bf16_peak},
+        "layer_roofline": {"t_roof_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms_per_step,
+                           "flops": l_flops, "bytes": l_bytes,
+                           "bound": "hbm" if l_bytes / (hbm * 1e9) >= l_flops / (bf16_peak * 1e12) else "tensor",
+                           "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained"},
+        "phases_ms": {p: float(np.mean(phase_ms[:, i])) for i, p in enumerate(moe.PHASES)},
+        "down_gemm": {"achieved_gbs": float(np.mean([x[1] for x in dn])) / (float(np.mean(dn_ms)) / 1000) / 1e9},
+        "rows_per_step": float(np.mean(kept_h.sum(1))),
+        "touched_experts": float(np.mean((kept_h > 0).sum(1))),
+        "max_vio": [round(float(v), 4) for v in vio_h[args.warmup:]],
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+        "gpu_launches": 10 * args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the cpu_baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per --impl reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = mi.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

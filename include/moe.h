@@ -1,0 +1,245 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of one sparse
+ * Mixture-of-Experts layer with shared experts, sigmoid or softmax routing,
+ * selection-only expert bias, optional group-limited top-K, optional capacity
+ * dropping, SwiGLU experts and the aux-loss-free bias step.
+ *
+ * The layer computed (notation of the source pages):
+ *
+ *   y_t = h_t + sum_{j=1..E_s} SwiGLU^S_j(h_t) + sum_{i in I_t} g_{t,i} SwiGLU^R_i(h_t)
+ *   SwiGLU(h) = (SiLU(h W_gate^T) * (h W_up^T)) W_down^T
+ *   s_{t,i} = sigmoid(h_t . e_i)             (score_fn = MOE_SCORE_SIGMOID)
+ *           = softmax_i(h_t . e_i)           (score_fn = MOE_SCORE_SOFTMAX, no bias)
+ *   I_t = TopK({s_{t,i} + b_i}, K)  [within the topk_groups best groups]
+ *   g_{t,i} = s_{t,i} / max(sum_{j in I_t} s_{t,j}, 1e-12)
+ *   b_i <- b_i + gamma * sign(c_bar - c_i),  c_i = #{t : i in I_t},  c_bar = K T / E_r
+ *   MaxVio = (max_i c_i - c_bar) / c_bar
+ *
+ * Sources: "Sparse Mixture-of-Experts (MoE): Routing Math, Load Balancing &
+ * Expert Parallelism" (section 0 layer equation; section 2 biased selection,
+ * unbiased gates and the sign step; section 3 capacity bound; section 4 MaxVio);
+ * "Mixture of Experts: Routing and Load Balancing" (section 2 routing rule;
+ * section 5 capacity admits tokens in order); "Load Balancing -- DeepSeek-V3"
+ * (How it works: g' and g; Official code: bias before grouped top-k);
+ * "GPUs, memory and failures" (worked bias example; the bias card).
+ *
+ * Conventions for every entry point
+ *  - Pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *    every buffer (inputs, outputs and the workspace `ws`).  The library never
+ *    allocates or frees device memory.  Arrays are dense, row-major, with no
+ *    padding; every device pointer must be 16-byte aligned.
+ *  - Activations and expert weights have the element type cfg->dtype
+ *    (MOE_DTYPE_F32: float; MOE_DTYPE_BF16: bfloat16 bits in uint16).
+ *    Centroids e, biases b, scores and gates are always float32; indices and
+ *    counts are int32.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *    enqueues work on it: no host synchronisation, no device->host copy.
+ *  - Errors: arguments are validated on the host first; on any failure the call
+ *    returns a non-zero moe_status and enqueues NOTHING
+ *    (moe_last_error_detail() describes the failure).  MOE_ERR_CUDA reports a
+ *    launch failure.  Faults the kernels detect themselves (a bounded wait that
+ *    expired, an index out of range) never trap: they set the error word held in
+ *    the workspace, read with moe_get_device_error() after the stream is
+ *    synchronised; the outputs of that call are then undefined.
+ *  - Shapes: d_model, d_ffn, d_ffn_shared must be multiples of 8 (16-byte
+ *    rows); 1 <= K <= min(E_r, 32); E_r <= 1024; E_s <= 8; T >= 1;
+ *    n_groups divides E_r; topk_groups * (E_r / n_groups) >= K; group_topn <=
+ *    E_r / n_groups.  Larger shapes return MOE_ERR_UNSUPPORTED.
+ *  - Determinism: for the same inputs every output is bitwise reproducible
+ *    (no floating-point atomics; every sum runs in a fixed order).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad shape or inconsistent config   */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement       */
+  MOE_ERR_WORKSPACE = 3,    /* ws is NULL, misaligned or smaller than required    */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed        */
+  MOE_ERR_DEVICE = 5        /* the device error word is set (moe_get_device_error)*/
+} moe_status;
+
+enum { MOE_SCORE_SIGMOID = 0, MOE_SCORE_SOFTMAX = 1 };
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+
+/* device error word values (moe_get_device_error) */
+enum {
+  MOE_DEVERR_NONE = 0,
+  MOE_DEVERR_WAIT_TIMEOUT = 1,   /* a pipeline barrier wait gave up (bounded spin) */
+  MOE_DEVERR_INDEX = 2           /* an expert index outside [0, E_r) was met       */
+};
+
+typedef struct {
+  int32_t T;             /* tokens in the batch (h is [T, d_model])                    */
+  int32_t d_model;       /* d                                                           */
+  int32_t E_r;           /* routed experts                                              */
+  int32_t E_s;           /* shared (always-on) experts, 0 allowed                       */
+  int32_t K;             /* experts selected per token                                  */
+  int32_t d_ffn;         /* routed expert width f                                       */
+  int32_t d_ffn_shared;  /* shared expert width f_s (ignored when E_s = 0)              */
+  int32_t score_fn;      /* MOE_SCORE_SIGMOID or MOE_SCORE_SOFTMAX                      */
+  int32_t n_groups;      /* expert groups for group-limited top-K (1 = no limit)        */
+  int32_t topk_groups;   /* groups kept per token                                       */
+  int32_t group_topn;    /* a group's score = sum of its top group_topn keys (0 = none) */
+  float capacity_factor; /* <= 0: dropless; else C = floor(T*K*CF/E_r) rows per expert  */
+  int32_t dtype;         /* MOE_DTYPE_F32 or MOE_DTYPE_BF16                             */
+  int32_t add_residual;  /* 1: y includes h_t                                           */
+} moe_config;
+
+/* Library ABI version (MOE_ABI_VERSION). */
+int32_t moe_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status s);
+
+/* Text describing the last failed validation in this thread (static buffer). */
+const char* moe_last_error_detail(void);
+
+/*
+ * Required workspace bytes for moe_layer_forward with this config (an upper
+ * bound for every other entry point with the same config).  *bytes is a HOST
+ * pointer.  The workspace must be 256-byte aligned device memory; its first
+ * 256 bytes hold the device error word, which the caller must zero once
+ * (cudaMemset) before first use.
+ */
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes);
+
+/*
+ * Router: affinity, selection and gates (steps a1-a4).
+ *   h      [T, d]   activations (cfg->dtype); may be NULL when s_in is given.
+ *   e      [E_r, d] float32 centroids; may be NULL when s_in is given.
+ *   b      [E_r]    float32 selection bias, or NULL for b = 0 (ignored for softmax).
+ *   s_in   [T, E_r] float32 scores to route from ("fed" mode: skips the affinity),
+ *                   or NULL to compute s from h and e (fp32 logits).
+ *   s_out  [T, E_r] float32: the scores used, or NULL.
+ *   idx    [T, K]   int32 out: I_t in ascending expert index.
+ *   gates  [T, K]   float32 out: g_{t,i} in the same order.
+ *   counts [E_r]    int32 out: c_i (before any capacity drop), or NULL.
+ * Selection keys are s + b in fp32; ties choose the lower expert (group) index.
+ * Sources: "Sparse Mixture-of-Experts ...", section 2 equation; "Load
+ * Balancing -- DeepSeek-V3", How it works / Official code.
+ */
+moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const float* b,
+                     const float* s_in, float* s_out, int32_t* idx, float* gates,
+                     int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dispatch: a stable permutation of the (token, slot) pairs grouped by expert
+ * (step a5).  Rows of expert i are offsets[i] .. offsets[i+1]-1, tokens ascending;
+ * with capacity, at most C = floor(T*K*CF/E_r) rows per expert (lowest token
+ * indices kept, "Sparse Mixture-of-Experts ...", section 3; "Mixture of
+ * Experts: Routing and Load Balancing", section 5).
+ *   idx      [T, K]      int32 in (from moe_route).
+ *   gates    [T, K]      float32 in, or NULL (then row_gate is not written).
+ *   h        [T, d]      activations, or NULL (then x_perm is not written).
+ *   offsets  [E_r + 1]   int32 out.        kept [E_r] int32 out (rows kept).
+ *   perm_tok [T*K]       int32 out: token of each row (first offsets[E_r] valid).
+ *   row_of   [T, K]      int32 out: row of (t, k), -1 when dropped.
+ *   row_gate [T*K]       float32 out: gate of each row, or NULL.
+ *   x_perm   [T*K, d]    out: h[perm_tok[r]] for each row, or NULL.
+ */
+moe_status moe_permute(const moe_config* cfg, const int32_t* idx, const float* gates,
+                       const void* h, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                       int32_t* kept, float* row_gate, void* x_perm, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Grouped SwiGLU experts (steps a6-a7) over expert-contiguous rows:
+ *   out[r] = row_scale[r] * SwiGLU_g(x[r])  for offsets[g] <= r < offsets[g+1].
+ *   n_experts    number of weight sets (groups); offsets is [n_experts + 1] on the
+ *                device; offsets[n_experts] <= max_rows (host-known bound).
+ *   d_ffn        expert width f (cfg->d_model is the model width d).
+ *   x            [max_rows, d];  w_gate, w_up [n_experts, f, d];  w_down [n_experts, d, f].
+ *   row_scale    [max_rows] float32, or NULL for 1.
+ *   out          [max_rows, d], cfg->dtype.  Rows >= offsets[n_experts] untouched.
+ * bf16 runs on the tensor cores (tcgen05, fp32 accumulation in TMEM; the SwiGLU
+ * product is rounded to bf16 before W_down); fp32 runs on CUDA cores in fp32.
+ */
+/* Workspace bytes moe_expert_ffn needs for these arguments (*bytes: HOST pointer). */
+moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,
+                                         int32_t max_rows, size_t* bytes);
+
+moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,
+                          int32_t max_rows, const int32_t* offsets, const void* x,
+                          const void* w_gate, const void* w_up, const void* w_down,
+                          const float* row_scale, void* out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Combine (step a8):  y_t = add_residual*h_t + sum_j shared_out[j, t]
+ *                           + sum_{k ascending, row_of[t,k] >= 0} slot[row_of[t,k]]
+ * accumulated in fp32 in exactly that order and rounded once to cfg->dtype.
+ *   slot       [rows, d]  gate-scaled routed expert outputs (cfg->dtype).
+ *   shared_out [E_s, T, d] shared expert outputs, or NULL when E_s = 0.
+ *   row_of     [T, K] int32.    y [T, d] out.
+ */
+moe_status moe_combine(const moe_config* cfg, const void* h, const void* slot,
+                       const void* shared_out, const int32_t* row_of, void* y, void* stream);
+
+/*
+ * Bias step (step a9), once per training step after the batch's loads are
+ * counted ("GPUs, memory and failures", the bias card; "Sparse
+ * Mixture-of-Experts ...", section 2):
+ *   b_i <- b_i + gamma * sign(K*T - E_r*c_i)   (sign(0) = 0; one fp32 add)
+ *   counts [E_r] int32 in;  b [E_r] float32 in/out;
+ *   max_vio: float32 device scalar out ((max c - c_bar)/c_bar), or NULL.
+ */
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float gamma, float* b,
+                           float* max_vio, void* stream);
+
+/*
+ * The whole layer (a1-a8, and a9 when update_bias != 0), on one stream with no
+ * host synchronisation.
+ *   h [T, d]; e [E_r, d] float32; b [E_r] float32 (read, and updated in place
+ *   when update_bias); w_gate/w_up [E_r, f, d], w_down [E_r, d, f];
+ *   ws_gate/ws_up [E_s, f_s, d], ws_down [E_s, d, f_s] (NULL when E_s = 0).
+ *   y [T, d] out.  Optional outputs (NULL to skip): idx_out [T, K],
+ *   gates_out [T, K], counts_out [E_r], kept_out [E_r], s_out [T, E_r],
+ *   max_vio_out (device float32 scalar; written whenever non-NULL).
+ *   s_in: optional fed scores [T, E_r] (skips the affinity; e may then be NULL).
+ * With update_bias, the routing of THIS call uses the incoming b and the step
+ * is applied afterwards (the bias is carried to the next step).
+ */
+moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* e, float* b,
+                             const void* w_gate, const void* w_up, const void* w_down,
+                             const void* ws_gate, const void* ws_up, const void* ws_down,
+                             const float* s_in, void* y, int32_t* idx_out, float* gates_out,
+                             int32_t* counts_out, int32_t* kept_out, float* s_out,
+                             int32_t update_bias, float gamma, float* max_vio_out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Profiling support.  When n_events > 0, every later moe_layer_forward call in
+ * this thread records the caller's CUDA events (cudaEvent_t handles, created
+ * and owned by the caller) on its stream at the phase boundaries:
+ *   0 start; 1 after routing (a1-a4); 2 after dispatch (a5); 3 after the FFN
+ *   group tables; 4 after the gate/up GEMM (a6); 5 after the down GEMM (a7);
+ *   6 after the combine (a8); 7 after the bias step (a9).
+ * Only the first n_events (<= 8) are recorded; n_events = 0 turns it off.
+ */
+moe_status moe_set_phase_events(void* const* events, int32_t n_events);
+
+/*
+ * Read (synchronously, via cudaMemcpy) the device error word of a workspace
+ * after the stream that used it has been synchronised.  *code is a HOST
+ * pointer.  Returns MOE_ERR_DEVICE when the word is non-zero, MOE_OK otherwise.
+ */
+moe_status moe_get_device_error(const void* ws, int32_t* code);
+
+/* Zero the device error word of a workspace (enqueued on stream). */
+moe_status moe_clear_device_error(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,426 @@
+// Host side of the C ABI declared in include/moe.h: argument validation,
+// workspace layout and the launch sequence of each entry point.  Every entry
+// point validates first and enqueues nothing on failure; none allocates.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+constexpr int kChunkShift = 8;          // histogram chunk = 256 tokens (the scatter block)
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t capacity_rows(const moe_config& c) {
+  const int64_t tk = (int64_t)c.T * c.K;
+  if (!(c.capacity_factor > 0.0f)) return tk;
+  double cap = std::floor((double)c.T * (double)c.K * (double)c.capacity_factor / (double)c.E_r);
+  if (cap > (double)tk) return tk;
+  return (int64_t)cap;
+}
+
+struct Layout {
+  size_t err, scores, hist, chunk_base, counts, kept, offsets, grp_rows, grp_row0, pre_gu, pre_dn;
+  size_t idx, gates, row_of, perm_tok, row_gate, maxvio, x_perm, act_r, act_s, slot_r, slot_s;
+  size_t total;
+  int n_chunks;
+  int64_t cap, R;
+};
+
+Layout make_layout(const moe_config& c) {
+  Layout L{};
+  const size_t es = elem_bytes(c.dtype);
+  const int G = c.E_r + c.E_s;
+  L.n_chunks = (c.T + (1 << kChunkShift) - 1) >> kChunkShift;
+  L.cap = capacity_rows(c);
+  int64_t R = std::min<int64_t>((int64_t)c.T * c.K, (int64_t)c.E_r * L.cap);
+  L.R = R < 1 ? 1 : R;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.err = take(kAlign);
+  L.scores = take((size_t)c.T * c.E_r * 4);
+  L.hist = take((size_t)L.n_chunks * c.E_r * 4);
+  L.chunk_base = take((size_t)L.n_chunks * c.E_r * 4);
+  L.counts = take((size_t)c.E_r * 4);
+  L.kept = take((size_t)c.E_r * 4);
+  L.offsets = take((size_t)(c.E_r + 1) * 4);
+  L.grp_rows = take((size_t)G * 4);
+  L.grp_row0 = take((size_t)G * 4);
+  L.pre_gu = take((size_t)(G + 1) * 4);
+  L.pre_dn = take((size_t)(G + 1) * 4);
+  L.idx = take((size_t)c.T * c.K * 4);
+  L.gates = take((size_t)c.T * c.K * 4);
+  L.row_of = take((size_t)c.T * c.K * 4);
+  L.perm_tok = take((size_t)L.R * 4);
+  L.row_gate = take((size_t)L.R * 4);
+  L.maxvio = take(4);
+  L.x_perm = take((size_t)L.R * c.d_model * es);
+  L.act_r = take((size_t)L.R * c.d_ffn * es);
+  L.act_s = take((size_t)c.E_s * c.T * (c.E_s ? c.d_ffn_shared : 0) * es);
+  L.slot_r = take((size_t)L.R * c.d_model * es);
+  L.slot_s = take((size_t)c.E_s * c.T * c.d_model * es);
+  L.total = o;
+  return L;
+}
+
+moe_status validate(const moe_config* cfg) {
+  if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  const moe_config& c = *cfg;
+  if (c.T < 1 || c.T > (1 << 24)) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [1, 2^24]", c.T);
+  if (c.d_model < 8 || c.d_model % 8) return fail(MOE_ERR_INVALID_ARG, "d_model=%d must be a positive multiple of 8", c.d_model);
+  if (c.E_r < 1) return fail(MOE_ERR_INVALID_ARG, "E_r=%d < 1", c.E_r);
+  if (c.E_r > 1024) return fail(MOE_ERR_UNSUPPORTED, "E_r=%d > 1024", c.E_r);
+  if (c.E_s < 0) return fail(MOE_ERR_INVALID_ARG, "E_s=%d < 0", c.E_s);
+  if (c.E_s > 8) return fail(MOE_ERR_UNSUPPORTED, "E_s=%d > 8", c.E_s);
+  if (c.K < 1 || c.K > c.E_r) return fail(MOE_ERR_INVALID_ARG, "K=%d outside [1, E_r=%d]", c.K, c.E_r);
+  if (c.K > 32) return fail(MOE_ERR_UNSUPPORTED, "K=%d > 32", c.K);
+  if (c.d_ffn < 8 || c.d_ffn % 8) return fail(MOE_ERR_INVALID_ARG, "d_ffn=%d must be a positive multiple of 8", c.d_ffn);
+  if (c.E_s > 0 && (c.d_ffn_shared < 8 || c.d_ffn_shared % 8))
+    return fail(MOE_ERR_INVALID_ARG, "d_ffn_shared=%d must be a positive multiple of 8", c.d_ffn_shared);
+  if (c.score_fn != MOE_SCORE_SIGMOID && c.score_fn != MOE_SCORE_SOFTMAX)
+    return fail(MOE_ERR_INVALID_ARG, "score_fn=%d", c.score_fn);
+  if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c.dtype);
+  if (c.add_residual != 0 && c.add_residual != 1) return fail(MOE_ERR_INVALID_ARG, "add_residual=%d", c.add_residual);
+  if (!std::isfinite(c.capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is not finite");
+  if (c.n_groups < 1) return fail(MOE_ERR_INVALID_ARG, "n_groups=%d < 1", c.n_groups);
+  if (c.group_topn < 0) return fail(MOE_ERR_INVALID_ARG, "group_topn=%d < 0", c.group_topn);
+  if (c.n_groups > 1 && c.group_topn > 0) {
+    if (c.E_r % c.n_groups) return fail(MOE_ERR_INVALID_ARG, "n_groups=%d does not divide E_r=%d", c.n_groups, c.E_r);
+    const int gsz = c.E_r / c.n_groups;
+    if (c.topk_groups < 1 || c.topk_groups > c.n_groups)
+      return fail(MOE_ERR_INVALID_ARG, "topk_groups=%d outside [1, n_groups=%d]", c.topk_groups, c.n_groups);
+    if ((int64_t)c.topk_groups * gsz < c.K)
+      return fail(MOE_ERR_INVALID_ARG, "topk_groups*(E_r/n_groups)=%d < K=%d", c.topk_groups * gsz, c.K);
+    if (c.group_topn > gsz) return fail(MOE_ERR_INVALID_ARG, "group_topn=%d > group size %d", c.group_topn, gsz);
+    if (c.n_groups > 32) return fail(MOE_ERR_UNSUPPORTED, "n_groups=%d > 32", c.n_groups);
+  }
+  if (c.dtype == MOE_DTYPE_BF16 && (c.d_model < 64 || c.d_ffn < 64 || (c.E_s > 0 && c.d_ffn_shared < 64)))
+    return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d_model, d_ffn, d_ffn_shared >= 64");
+  return MOE_OK;
+}
+
+moe_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "ws is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(MOE_ERR_WORKSPACE, "ws is not 256-byte aligned");
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "ws_bytes=%zu < required %zu", ws_bytes, need);
+  return MOE_OK;
+}
+
+moe_status cuda_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "CUDA error: %s", cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+#define MOE_CHECK(x) do { moe_status s_ = (x); if (s_ != MOE_OK) return s_; } while (0)
+#define MOE_NONNULL(p) do { if (!(p)) return fail(MOE_ERR_INVALID_ARG, #p " is NULL"); \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, #p " is not 16-byte aligned"); } while (0)
+#define MOE_ALIGNED(p) do { if ((p) && !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, #p " is not 16-byte aligned"); } while (0)
+
+template <typename T> T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+bool use_tensor_cores(int dtype) { return dtype == MOE_DTYPE_BF16; }
+
+// Caller-provided CUDA events recorded at the phase boundaries of
+// moe_layer_forward (profiling support; see moe_set_phase_events).
+thread_local cudaEvent_t g_phase_events[8] = {};
+thread_local int g_n_phase_events = 0;
+
+void mark_phase(int i, cudaStream_t st) {
+  if (i < g_n_phase_events && g_phase_events[i]) cudaEventRecord(g_phase_events[i], st);
+}
+
+// Group tables + both GEMMs of the grouped FFN (phase marks 3 and 4 after the
+// group tables and the gate/up GEMM when phase_base >= 0).
+moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int max_rows,
+                   cudaStream_t st, int phase_base = -1) {
+  const bool tc = use_tensor_cores(c.dtype);
+  const int bm = tc ? moe::tc_bm() : moe::simt_bm();
+  const int bn_gu = tc ? moe::tc_cols_gateup() : moe::simt_bn();
+  const int bn_dn = tc ? moe::tc_cols_down() : moe::simt_bn();
+  moe::launch_groups(offsets, a.E_r, a.E_s, a.T, bm, (a.f_r + bn_gu - 1) / bn_gu,
+                     a.E_s ? (a.f_s + bn_gu - 1) / bn_gu : 0, (a.d + bn_dn - 1) / bn_dn,
+                     (a.d + bn_dn - 1) / bn_dn, const_cast<int*>(a.grp_rows),
+                     const_cast<int*>(a.grp_row0), const_cast<int*>(a.pre_gu),
+                     const_cast<int*>(a.pre_dn), max_rows, a.err, st);
+  if (phase_base >= 0) mark_phase(phase_base, st);
+  for (int which = 0; which < 2; ++which) {
+    if (tc) {
+      cudaError_t e = moe::launch_ffn_tc(a, which, st);
+      if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "tensor-core FFN launch: %s", cudaGetErrorString(e));
+    } else {
+      moe::launch_ffn_simt(a, which, st);
+    }
+    if (phase_base >= 0 && which == 0) mark_phase(phase_base + 1, st);
+  }
+  return cuda_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_error_detail(void) { return g_detail; }
+
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes) {
+  MOE_CHECK(validate(cfg));
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = make_layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,
+                                         int32_t max_rows, size_t* bytes) {
+  MOE_CHECK(validate(cfg));
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_experts < 1 || n_experts > 1024) return fail(MOE_ERR_INVALID_ARG, "n_experts=%d outside [1, 1024]", n_experts);
+  if (d_ffn < 8 || d_ffn % 8) return fail(MOE_ERR_INVALID_ARG, "d_ffn=%d must be a positive multiple of 8", d_ffn);
+  if (max_rows < 0) return fail(MOE_ERR_INVALID_ARG, "max_rows=%d < 0", max_rows);
+  size_t o = 0;
+  o = align_up(o + kAlign);                                  // error word
+  o = align_up(o + (size_t)n_experts * 8);                    // grp_rows, grp_row0
+  o = align_up(o + (size_t)(n_experts + 1) * 8);              // pre_gu, pre_dn
+  o = align_up(o + (size_t)(max_rows < 1 ? 1 : max_rows) * d_ffn * elem_bytes(cfg->dtype));
+  *bytes = o;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const float* b,
+                     const float* s_in, float* s_out, int32_t* idx, float* gates,
+                     int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  if (!s_in) { MOE_NONNULL(h); MOE_NONNULL(e); }
+  MOE_ALIGNED(s_in); MOE_ALIGNED(s_out); MOE_ALIGNED(b); MOE_ALIGNED(counts);
+  MOE_NONNULL(idx); MOE_NONNULL(gates);
+  const Layout L = make_layout(c);
+  MOE_CHECK(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* hist = at<int>(ws, L.hist);
+  float* scores = at<float>(ws, L.scores);
+  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
+  if (!s_in) moe::launch_router_logits(h, c.dtype, e, scores, c.T, c.d_model, c.E_r, st);
+  moe::launch_select(s_in ? s_in : scores, s_in != nullptr,
+                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
+                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
+  if (counts) moe::launch_counts(hist, L.n_chunks, c.E_r, counts, st);
+  return cuda_status();
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* idx, const float* gates,
+                       const void* h, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                       int32_t* kept, float* row_gate, void* x_perm, void* ws, size_t ws_bytes,
+                       void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  MOE_NONNULL(idx); MOE_NONNULL(offsets); MOE_NONNULL(perm_tok); MOE_NONNULL(row_of); MOE_NONNULL(kept);
+  MOE_ALIGNED(gates); MOE_ALIGNED(h); MOE_ALIGNED(row_gate); MOE_ALIGNED(x_perm);
+  if (row_gate && !gates) return fail(MOE_ERR_INVALID_ARG, "row_gate needs gates");
+  if (x_perm && !h) return fail(MOE_ERR_INVALID_ARG, "x_perm needs h");
+  const Layout L = make_layout(c);
+  MOE_CHECK(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err = at<int>(ws, L.err);
+  int* hist = at<int>(ws, L.hist);
+  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
+  moe::launch_hist(idx, hist, kChunkShift, c.T, c.K, c.E_r, err, st);
+  moe::launch_scan(hist, L.n_chunks, c.E_r, (int)L.cap, at<int>(ws, L.counts), kept, offsets,
+                   at<int>(ws, L.chunk_base), st);
+  moe::launch_scatter(idx, gates, offsets, at<int>(ws, L.chunk_base), (int)L.cap, c.T, c.K, c.E_r,
+                      perm_tok, row_of, row_gate, err, st);
+  if (x_perm)
+    moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model, (int)elem_bytes(c.dtype),
+                       c.T * c.K, c.T, err, st);
+  return cuda_status();
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,
+                          int32_t max_rows, const int32_t* offsets, const void* x,
+                          const void* w_gate, const void* w_up, const void* w_down,
+                          const float* row_scale, void* out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  size_t need = 0;
+  MOE_CHECK(moe_expert_ffn_workspace_size(cfg, n_experts, d_ffn, max_rows, &need));
+  const moe_config& c = *cfg;
+  if (c.dtype == MOE_DTYPE_BF16 && d_ffn < 64) return fail(MOE_ERR_UNSUPPORTED, "bf16 needs d_ffn >= 64");
+  MOE_NONNULL(offsets); MOE_NONNULL(x); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down);
+  MOE_NONNULL(out); MOE_ALIGNED(row_scale);
+  MOE_CHECK(check_ws(ws, ws_bytes, need));
+  if (max_rows == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  size_t o = kAlign;
+  int* grp_rows = at<int>(ws, o);
+  int* grp_row0 = grp_rows + n_experts;
+  o = align_up(o + (size_t)n_experts * 8);
+  int* pre_gu = at<int>(ws, o);
+  int* pre_dn = pre_gu + n_experts + 1;
+  o = align_up(o + (size_t)(n_experts + 1) * 8);
+  moe::FfnArgs a{};
+  a.dtype = c.dtype; a.T = c.T; a.d = c.d_model; a.f_r = d_ffn; a.f_s = d_ffn;
+  a.E_r = n_experts; a.E_s = 0; a.max_rows_r = max_rows;
+  a.x_r = x; a.x_s = x;
+  a.wg_r = w_gate; a.wu_r = w_up; a.wd_r = w_down;
+  a.wg_s = w_gate; a.wu_s = w_up; a.wd_s = w_down;
+  a.grp_rows = grp_rows; a.grp_row0 = grp_row0; a.pre_gu = pre_gu; a.pre_dn = pre_dn;
+  a.row_scale = row_scale;
+  a.act_r = at<void>(ws, o); a.act_s = a.act_r;
+  a.out_r = out; a.out_s = out;
+  a.err = at<int>(ws, 0);
+  return run_ffn(c, a, offsets, max_rows, st);
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* h, const void* slot,
+                       const void* shared_out, const int32_t* row_of, void* y, void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  MOE_NONNULL(h); MOE_NONNULL(slot); MOE_NONNULL(row_of); MOE_NONNULL(y);
+  if (c.E_s > 0) MOE_NONNULL(shared_out);
+  moe::launch_combine(h, slot, shared_out, row_of, y, c.T, c.d_model, c.K, c.E_s, c.add_residual,
+                      c.dtype, 0x7FFFFFFF, static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float gamma, float* b,
+                           float* max_vio, void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  MOE_NONNULL(counts); MOE_NONNULL(b);
+  if (!std::isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not finite");
+  moe::launch_bias_update(counts, b, gamma, max_vio, c.E_r, c.K, c.T, static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* e, float* b,
+                             const void* w_gate, const void* w_up, const void* w_down,
+                             const void* ws_gate, const void* ws_up, const void* ws_down,
+                             const float* s_in, void* y, int32_t* idx_out, float* gates_out,
+                             int32_t* counts_out, int32_t* kept_out, float* s_out,
+                             int32_t update_bias, float gamma, float* max_vio_out,
+                             void* ws, size_t ws_bytes, void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  MOE_NONNULL(h); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down); MOE_NONNULL(y);
+  if (!s_in) MOE_NONNULL(e);
+  if (c.E_s > 0) { MOE_NONNULL(ws_gate); MOE_NONNULL(ws_up); MOE_NONNULL(ws_down); }
+  if (update_bias) {
+    MOE_NONNULL(b);
+    if (!std::isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not finite");
+  }
+  MOE_ALIGNED(b); MOE_ALIGNED(s_in); MOE_ALIGNED(idx_out); MOE_ALIGNED(gates_out);
+  MOE_ALIGNED(counts_out); MOE_ALIGNED(kept_out); MOE_ALIGNED(s_out); MOE_ALIGNED(max_vio_out);
+  const Layout L = make_layout(c);
+  MOE_CHECK(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int* err = at<int>(ws, L.err);
+  int* hist = at<int>(ws, L.hist);
+  float* scores = at<float>(ws, L.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+  float* gates = gates_out ? gates_out : at<float>(ws, L.gates);
+  int* counts = counts_out ? counts_out : at<int>(ws, L.counts);
+  int* kept = kept_out ? kept_out : at<int>(ws, L.kept);
+  int* offsets = at<int>(ws, L.offsets);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  int32_t* perm_tok = at<int32_t>(ws, L.perm_tok);
+  float* row_gate = at<float>(ws, L.row_gate);
+  const size_t es = elem_bytes(c.dtype);
+
+  // a1-a4: affinity, selection, gates, per-chunk histogram
+  mark_phase(0, st);
+  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
+  if (!s_in) moe::launch_router_logits(h, c.dtype, e, scores, c.T, c.d_model, c.E_r, st);
+  moe::launch_select(s_in ? s_in : scores, s_in != nullptr,
+                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
+                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
+  // a5: counts, capacity, offsets, stable scatter, row gather
+  mark_phase(1, st);
+  moe::launch_scan(hist, L.n_chunks, c.E_r, (int)L.cap, counts, kept, offsets,
+                   at<int>(ws, L.chunk_base), st);
+  moe::launch_scatter(idx, gates, offsets, at<int>(ws, L.chunk_base), (int)L.cap, c.T, c.K, c.E_r,
+                      perm_tok, row_of, row_gate, err, st);
+  void* x_perm = at<void>(ws, L.x_perm);
+  moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model, (int)es, (int)L.R, c.T, err, st);
+  mark_phase(2, st);
+  // a6-a7: grouped SwiGLU experts (routed + shared) with gate-scaled outputs
+  moe::FfnArgs a{};
+  a.dtype = c.dtype; a.T = c.T; a.d = c.d_model; a.f_r = c.d_ffn;
+  a.f_s = c.E_s ? c.d_ffn_shared : c.d_ffn;
+  a.E_r = c.E_r; a.E_s = c.E_s; a.max_rows_r = (int)L.R;
+  a.x_r = x_perm; a.x_s = h;
+  a.wg_r = w_gate; a.wu_r = w_up; a.wd_r = w_down;
+  a.wg_s = c.E_s ? ws_gate : w_gate; a.wu_s = c.E_s ? ws_up : w_up; a.wd_s = c.E_s ? ws_down : w_down;
+  a.grp_rows = at<int>(ws, L.grp_rows); a.grp_row0 = at<int>(ws, L.grp_row0);
+  a.pre_gu = at<int>(ws, L.pre_gu); a.pre_dn = at<int>(ws, L.pre_dn);
+  a.row_scale = row_gate;
+  a.act_r = at<void>(ws, L.act_r); a.act_s = c.E_s ? at<void>(ws, L.act_s) : a.act_r;
+  a.out_r = at<void>(ws, L.slot_r); a.out_s = c.E_s ? at<void>(ws, L.slot_s) : a.out_r;
+  a.err = err;
+  MOE_CHECK(run_ffn(c, a, offsets, (int)L.R, st, 3));
+  mark_phase(5, st);
+  // a8: fixed-order combine with the residual
+  moe::launch_combine(h, a.out_r, c.E_s ? a.out_s : nullptr, row_of, y, c.T, c.d_model, c.K, c.E_s,
+                      c.add_residual, c.dtype, (int)L.R, st);
+  mark_phase(6, st);
+  // a9: the bias step, after this batch's loads are counted
+  if (update_bias || max_vio_out)
+    moe::launch_bias_update(counts, update_bias ? b : nullptr, gamma, max_vio_out, c.E_r, c.K, c.T, st);
+  mark_phase(7, st);
+  return cuda_status();
+}
+
+moe_status moe_set_phase_events(void* const* events, int32_t n_events) {
+  if (n_events < 0 || n_events > 8) return fail(MOE_ERR_INVALID_ARG, "n_events=%d outside [0, 8]", n_events);
+  if (n_events > 0 && !events) return fail(MOE_ERR_INVALID_ARG, "events is NULL");
+  for (int i = 0; i < 8; ++i) g_phase_events[i] = i < n_events ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  g_n_phase_events = n_events;
+  return MOE_OK;
+}
+
+moe_status moe_get_device_error(const void* ws, int32_t* code) {
+  if (!ws || !code) return fail(MOE_ERR_INVALID_ARG, "ws or code is NULL");
+  int32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_status();
+  *code = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+moe_status moe_clear_device_error(void* ws, void* stream) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "ws is NULL");
+  cudaMemsetAsync(ws, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,385 @@
+// Grouped SwiGLU experts on the 5th-generation tensor cores (sm_100a):
+// tcgen05.mma with bf16 operands staged in shared memory by TMA and fp32
+// accumulators in tensor memory (TMEM), one persistent CTA per SM.
+//
+//   gate/up GEMM:  D = X W_gate^T | X W_up^T      epilogue: act = SiLU(gate) * up -> bf16
+//   down GEMM:     D = act W_down^T                epilogue: out = g_{t,i} * D     -> bf16
+//
+// SwiGLU(h) = (SiLU(h W_gate^T) * (h W_up^T)) W_down^T and the gate-weighted
+// routed sum follow "Sparse Mixture-of-Experts (MoE): Routing Math, Load
+// Balancing & Expert Parallelism" (section 0 layer equation; section 3 "a
+// single fused Grouped GEMM over variable-sized token buckets").
+//
+// Work unit = (group, 128-row tile, 256-column B tile).  Groups are the routed
+// experts (expert-contiguous rows of the permuted activations) followed by the
+// shared experts (all T tokens); the unit -> group map is a device-side prefix
+// sum, so per-expert row counts never travel to the host.  Units are ordered
+// row-tile fastest, so the CTAs running at the same time share weight tiles
+// through L2 and each expert's weights stream from HBM about once.
+//
+// Warp roles (192 threads): warp 0 = TMA producer (+ TMEM allocation), warp 1 =
+// MMA issuer (one thread), warps 2..5 = epilogue (TMEM -> registers -> global).
+// Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the
+// epilogue of one unit overlaps the MMAs of the next.
+#include <cuda.h>
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;                         // rows per tile (MMA M)
+constexpr int BN = 256;                         // B rows per tile (MMA N)
+constexpr int BK = 64;                          // K per stage: one 128-byte swizzle atom of bf16
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
+
+struct Params {
+  CUtensorMap a_r, a_s;       // A: routed rows / shared rows
+  CUtensorMap b0_r, b1_r;     // routed B: gate & up (SWIGLU) or down (b0 only)
+  CUtensorMap b0_s, b1_s;     // shared B
+  const int* grp_rows;
+  const int* grp_row0;
+  const int* prefix;          // [G + 1] unit prefix
+  int G, E_r;
+  int k_r, k_s;               // reduction length (routed / shared)
+  int wrows_r, wrows_s;       // B rows per expert in the stacked weight tensors
+  int ncols_r, ncols_s;       // output columns
+  uint16_t* out_r;
+  uint16_t* out_s;
+  const float* row_scale;     // routed rows' gates (EPI_SCALE), may be null
+  int* err;
+};
+
+__device__ __forceinline__ void decode(const Params& p, int u, int& g, int& mt, int& nt) {
+  int lo = 0, hi = p.G;
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(p.prefix + mid) <= u) lo = mid; else hi = mid;
+  }
+  g = lo;
+  int local = u - __ldg(p.prefix + g);
+  int mtiles = (__ldg(p.grp_rows + g) + BM - 1) / BM;
+  mt = local % mtiles;
+  nt = local / mtiles;
+}
+
+// Wait without giving up on *abort (used to drain copies and MMAs in flight
+// before the CTA releases its shared and tensor memory).
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int* err) {
+  uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) { set_device_error(err, MOE_DEVERR_WAIT_TIMEOUT); return; }
+  }
+}
+
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4 * kWarp); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.b0_r);
+    prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = __ldg(p.prefix + p.G);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        int g, mt, nt;
+        decode(p, u, g, mt, nt);
+        const bool sh = g >= p.E_r;
+        const int e = sh ? g - p.E_r : g;
+        const CUtensorMap* am = sh ? &p.a_s : &p.a_r;
+        const int arow = ((EPI == EPI_SWIGLU && sh) ? 0 : __ldg(p.grp_row0 + g)) + mt * BM;
+        const int wrows = sh ? p.wrows_s : p.wrows_r;
+        const int brow = e * wrows + nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
+        const CUtensorMap* b0 = sh ? &p.b0_s : &p.b0_r;
+        const CUtensorMap* b1 = sh ? &p.b1_s : &p.b1_r;
+        const int nk = ((sh ? p.k_s : p.k_r) + BK - 1) / BK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, am, &full[stage], kb * BK, arow);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(sB + stage * B_BYTES, b0, &full[stage], kb * BK, brow);
+            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, b1, &full[stage], kb * BK, brow);
+          } else {
+            tma_load_2d(sB + stage * B_BYTES, b0, &full[stage], kb * BK, brow);
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    producer_done:
+      // the last (up to STAGES) loads must have landed before shared memory is released
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--stage < 0) { stage = STAGES - 1; phase ^= 1u; }
+        wait_drain(&full[stage], phase, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        int g, mt, nt;
+        decode(p, u, g, mt, nt);
+        const bool sh = g >= p.E_r;
+        const int nk = ((sh ? p.k_s : p.k_r) + BK - 1) / BK;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2),
+                        sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), IDESC, (kb | k) != 0);
+          }
+          tc_commit(&empty[stage]);       // frees the stage once these MMAs are done
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);        // accumulator ready for the epilogue
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      tc_commit(drain);                    // every MMA issued by this thread is done
+      wait_drain(drain, 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int sub = warp & 3;              // TMEM lane quarter this warp may access
+    const int r = sub * 32 + lane;         // row within the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      int g, mt, nt;
+      decode(p, u, g, mt, nt);
+      const bool sh = g >= p.E_r;
+      const int rows = __ldg(p.grp_rows + g);
+      const int m = mt * BM + r;
+      const bool valid = m < rows;
+      const size_t orow = (size_t)__ldg(p.grp_row0 + g) + m;
+      const int ncols = sh ? p.ncols_s : p.ncols_r;
+      uint16_t* out = (sh ? p.out_s : p.out_r) + orow * ncols;
+      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          float gv[32], uv[32];
+          tmem_ld32(tb + c, gv);
+          tmem_ld32(tb + BN / 2 + c, uv);
+          const int col0 = nt * (BN / 2) + c;
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col0 + 8 * v < ncols) {
+                uint4 pk;
+                pk.x = pack_bf16(silu(gv[8 * v + 0]) * uv[8 * v + 0], silu(gv[8 * v + 1]) * uv[8 * v + 1]);
+                pk.y = pack_bf16(silu(gv[8 * v + 2]) * uv[8 * v + 2], silu(gv[8 * v + 3]) * uv[8 * v + 3]);
+                pk.z = pack_bf16(silu(gv[8 * v + 4]) * uv[8 * v + 4], silu(gv[8 * v + 5]) * uv[8 * v + 5]);
+                pk.w = pack_bf16(silu(gv[8 * v + 6]) * uv[8 * v + 6], silu(gv[8 * v + 7]) * uv[8 * v + 7]);
+                *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
+              }
+            }
+          }
+        }
+      } else {
+        const float scale = (!sh && p.row_scale && valid) ? __ldg(p.row_scale + orow) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float dv[32];
+          tmem_ld32(tb + c, dv);
+          const int col0 = nt * BN + c;
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col0 + 8 * v < ncols) {
+                uint4 pk;
+                pk.x = pack_bf16(dv[8 * v + 0] * scale, dv[8 * v + 1] * scale);
+                pk.y = pack_bf16(dv[8 * v + 2] * scale, dv[8 * v + 3] * scale);
+                pk.z = pack_bf16(dv[8 * v + 4] * scale, dv[8 * v + 5] * scale);
+                pk.w = pack_bf16(dv[8 * v + 6] * scale, dv[8 * v + 7] * scale);
+                *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows, cols] row-major (cols contiguous), box = 64 cols x box_rows
+static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+int tc_bm() { return tc::BM; }
+int tc_cols_gateup() { return tc::BN / 2; }
+int tc_cols_down() { return tc::BN; }
+
+static int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
+  using namespace tc;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    attr_done[dev] = true;
+  }
+  const bool has_s = a.E_s > 0;
+  Params p{};
+  bool ok = true;
+  p.grp_rows = a.grp_rows;
+  p.grp_row0 = a.grp_row0;
+  p.G = a.E_r + a.E_s;
+  p.E_r = a.E_r;
+  p.err = a.err;
+  if (which == 0) {
+    // gate/up: A = permuted tokens (routed) or h (shared); B = gate | up, 128 rows each
+    const uint64_t wr_r = (uint64_t)a.E_r * a.f_r, wr_s = has_s ? (uint64_t)a.E_s * a.f_s : wr_r;
+    ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM);
+    ok &= make_tmap(&p.a_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d, BM);
+    ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, BN / 2);
+    ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, BN / 2);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, BN / 2);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wu_s : a.wu_r, wr_s, a.d, BN / 2);
+    p.prefix = a.pre_gu;
+    p.k_r = p.k_s = a.d;
+    p.wrows_r = a.f_r; p.wrows_s = a.f_s;
+    p.ncols_r = a.f_r; p.ncols_s = a.f_s;
+    p.out_r = (uint16_t*)a.act_r; p.out_s = (uint16_t*)a.act_s;
+    p.row_scale = nullptr;
+  } else {
+    // down: A = act (routed / shared); B = W_down, 256 rows
+    const uint64_t rows_s = has_s ? (uint64_t)a.E_s * a.T : (uint64_t)a.max_rows_r;
+    const int fs = has_s ? a.f_s : a.f_r;
+    const uint64_t wd_rows_s = (uint64_t)(has_s ? a.E_s : a.E_r) * a.d;
+    ok &= make_tmap(&p.a_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, BM);
+    ok &= make_tmap(&p.a_s, has_s ? a.act_s : a.act_r, rows_s, fs, BM);
+    ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
+    ok &= make_tmap(&p.b1_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN);
+    p.prefix = a.pre_dn;
+    p.k_r = a.f_r; p.k_s = a.f_s;
+    p.wrows_r = a.d; p.wrows_s = a.d;
+    p.ncols_r = a.d; p.ncols_s = a.d;
+    p.out_r = (uint16_t*)a.out_r; p.out_s = (uint16_t*)a.out_s;
+    p.row_scale = a.row_scale;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const int grid = num_sms();
+  if (which == 0)
+    grouped_gemm_kernel<EPI_SWIGLU><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  else
+    grouped_gemm_kernel<EPI_SCALE><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

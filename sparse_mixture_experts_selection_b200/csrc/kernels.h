@@ -1,0 +1,56 @@
+// Internal launchers of the MoE library (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Arguments of the grouped SwiGLU FFN over routed groups (rows
+// grp_row0[g] .. +grp_rows[g] of x_r / act_r / out_r, weights of expert g) and
+// shared groups (all T rows of x_s, rows j*T.. of act_s / out_s).
+struct FfnArgs {
+  int dtype, T, d, f_r, f_s, E_r, E_s, max_rows_r;
+  const void *x_r, *x_s;
+  const void *wg_r, *wu_r, *wd_r, *wg_s, *wu_s, *wd_s;
+  const int *grp_rows, *grp_row0, *pre_gu, *pre_dn;
+  const float* row_scale;
+  void *act_r, *act_s, *out_r, *out_s;
+  int* err;
+};
+
+void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
+                          cudaStream_t st);
+void launch_select(const float* in, int in_is_scores, const float* bias, int score_fn,
+                   float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
+                   int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st);
+void launch_hist(const int32_t* idx, int* hist, int chunk_shift, int T, int K, int E, int* err,
+                 cudaStream_t st);
+void launch_counts(const int* hist, int n_chunks, int E, int* counts, cudaStream_t st);
+void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int* kept,
+                 int* offsets, int* chunk_base, cudaStream_t st);
+void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
+                   int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
+                   int* pre_dn, int max_rows, int* err, cudaStream_t st);
+void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
+                    const int* chunk_base, int cap, int T, int K, int E, int32_t* perm_tok,
+                    int32_t* row_of, float* row_gate, int* err, cudaStream_t st);
+void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
+                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st);
+void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
+                    void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
+                    int n_slot_rows, cudaStream_t st);
+void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
+                        int T, cudaStream_t st);
+
+int simt_bm();
+int simt_bn();
+void launch_ffn_simt(const FfnArgs& a, int which, cudaStream_t st);
+
+int tc_bm();
+int tc_cols_gateup();
+int tc_cols_down();
+// which = 0: gate/up GEMM + SwiGLU epilogue; which = 1: down GEMM + gate scaling
+cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st);
+
+}  // namespace moe

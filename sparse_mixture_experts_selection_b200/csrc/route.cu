@@ -1,0 +1,571 @@
+// Routing, dispatch, combine and bias-step kernels of the MoE layer forward.
+//
+// Sources (web pages):
+//  "Sparse Mixture-of-Experts (MoE): Routing Math, Load Balancing & Expert
+//   Parallelism": section 0 layer equation (combine), section 2 equation
+//   (I_t = TopK(s + b), g = s / sum s, c_i, c_bar, b += gamma sign(c_bar - c_i)),
+//   section 3 capacity bound, section 4 MaxVio.
+//  "Load Balancing -- DeepSeek-V3": How it works (g', g); Official code
+//   (bias added before the grouped top-k).
+//  "Mixture of Experts: Routing and Load Balancing": section 5 (capacity admits
+//   tokens in the order they appear).
+//  "GPUs, memory and failures": the bias card (update once per step).
+#include <cfloat>
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// a1 (CUDA cores): z[t, i] = sum_k h[t, k] e[i, k] in fp32.
+// Tile 64 tokens x 64 experts x 32 k, 256 threads, 4 x 4 outputs per thread.
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+router_logits_simt_kernel(const TIn* __restrict__ h, const float* __restrict__ e,
+                          float* __restrict__ z, int T, int d, int E) {
+  constexpr int BT = 64, BE = 64, BK = 32;
+  __shared__ float hs[BK][BT + 4];
+  __shared__ float es[BK][BE + 4];
+  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * BE;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += BK) {
+    for (int i = tid; i < BT * BK; i += 256) {
+      int r = i / BK, c = i % BK;
+      int t = t0 + r, k = k0 + c;
+      hs[c][r] = (t < T && k < d) ? to_f32(h[(size_t)t * d + k]) : 0.f;
+      int ex = e0 + r;
+      es[c][r] = (ex < E && k < d) ? e[(size_t)ex * d + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < BK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = hs[k][ty * 4 + i]; b[i] = es[k][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int ex = e0 + tx * 4 + j;
+      if (ex < E) z[(size_t)t * E + ex] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a1-a4: scores, (group-limited) top-K, gates and the per-chunk histogram.
+// One warp per token; lane l holds experts l, l+32, ... (KPL per lane).
+// ---------------------------------------------------------------------------
+
+// (key, index) order of the selection: larger key first, ties -> lower index.
+__device__ __forceinline__ bool beats(float ka, int ia, float kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+
+__device__ __forceinline__ void warp_best(float& k, int& i) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float ok = __shfl_xor_sync(kFull, k, off);
+    int oi = __shfl_xor_sync(kFull, i, off);
+    if (beats(ok, oi, k, i)) { k = ok; i = oi; }
+  }
+}
+
+template <int KPL>
+__global__ void __launch_bounds__(256)
+select_kernel(const float* __restrict__ in, int in_is_scores, const float* __restrict__ bias,
+              int score_fn, float* __restrict__ s_out, int32_t* __restrict__ idx,
+              float* __restrict__ gates, int* __restrict__ hist, int chunk_shift, int T, int E,
+              int K, int n_groups, int topk_groups, int group_topn) {
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
+  if (t >= T) return;
+  const float* row = in + (size_t)t * E;
+
+  float s[KPL], key[KPL];
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    int ex = j * kWarp + lane;
+    s[j] = ex < E ? row[ex] : 0.f;
+  }
+  if (!in_is_scores) {
+    if (score_fn == MOE_SCORE_SIGMOID) {
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) s[j] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-s[j])));
+    } else {
+      float m = -FLT_MAX;
+#pragma unroll
+      for (int j = 0; j < KPL; ++j)
+        if (j * kWarp + lane < E) m = fmaxf(m, s[j]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) {
+        s[j] = (j * kWarp + lane < E) ? expf(s[j] - m) : 0.f;
+        sum = __fadd_rn(sum, s[j]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(kFull, sum, off));
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) s[j] = __fdiv_rn(s[j], sum);
+    }
+  }
+  if (s_out) {
+#pragma unroll
+    for (int j = 0; j < KPL; ++j)
+      if (j * kWarp + lane < E) s_out[(size_t)t * E + j * kWarp + lane] = s[j];
+  }
+  // selection key: s + b as one fp32 add (the bias only picks)
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    int ex = j * kWarp + lane;
+    key[j] = ex < E ? __fadd_rn(s[j], bias ? bias[ex] : 0.0f) : -INFINITY;
+  }
+
+  // group limit: keep the topk_groups groups with the largest sum of their
+  // group_topn largest keys (added in descending order); others ineligible
+  uint32_t eligible = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j)
+    if (j * kWarp + lane < E) eligible |= 1u << j;
+  if (n_groups > 1 && group_topn > 0) {
+    const int gsz = E / n_groups;
+    float G[32];
+    for (int g = 0; g < n_groups; ++g) {
+      uint32_t used = 0;
+      float acc = 0.f;
+      for (int r = 0; r < group_topn; ++r) {
+        float bk = -INFINITY;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+          int ex = j * kWarp + lane;
+          if (ex < E && ex / gsz == g && !(used >> j & 1u) && beats(key[j], ex, bk, bi)) {
+            bk = key[j];
+            bi = ex;
+          }
+        }
+        warp_best(bk, bi);
+        if ((bi & (kWarp - 1)) == lane) used |= 1u << (bi / kWarp);
+        acc = r == 0 ? bk : __fadd_rn(acc, bk);
+      }
+      G[g] = acc;
+    }
+    uint32_t keep = 0;
+    for (int r = 0; r < topk_groups; ++r) {
+      int bg = -1;
+      for (int g = 0; g < n_groups; ++g)
+        if (!(keep >> g & 1u) && (bg < 0 || G[g] > G[bg])) bg = g;
+      keep |= 1u << bg;
+    }
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      int ex = j * kWarp + lane;
+      if (ex < E && !(keep >> (ex / gsz) & 1u)) eligible &= ~(1u << j);
+    }
+  }
+
+  // top-K among the eligible experts
+  uint32_t taken = 0;
+  for (int r = 0; r < K; ++r) {
+    float bk = -INFINITY;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      int ex = j * kWarp + lane;
+      if ((eligible >> j & 1u) && !(taken >> j & 1u) && beats(key[j], ex, bk, bi)) {
+        bk = key[j];
+        bi = ex;
+      }
+    }
+    warp_best(bk, bi);
+    if ((bi & (kWarp - 1)) == lane) taken |= 1u << (bi / kWarp);
+  }
+
+  // gate denominator: sum of the selected s in ascending expert index, fp32
+  float S = 0.f;
+  bool first = true;
+  int pos_of[KPL];
+  int pos = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    uint32_t m = __ballot_sync(kFull, taken >> j & 1u);
+    pos_of[j] = pos + __popc(m & ((1u << lane) - 1u));
+    pos += __popc(m);
+    while (m) {
+      int l = __ffs(m) - 1;
+      float v = __shfl_sync(kFull, s[j], l);
+      S = first ? v : __fadd_rn(S, v);
+      first = false;
+      m &= m - 1;
+    }
+  }
+  const float denom = fmaxf(S, 1e-12f);
+  const int chunk = t >> chunk_shift;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    if (taken >> j & 1u) {
+      int ex = j * kWarp + lane;
+      idx[(size_t)t * K + pos_of[j]] = ex;
+      gates[(size_t)t * K + pos_of[j]] = __fdiv_rn(s[j], denom);
+      if (hist) atomicAdd(&hist[(size_t)chunk * E + ex], 1);
+    }
+  }
+}
+
+// Histogram of a given idx [T, K] per chunk of tokens (for moe_permute).
+__global__ void hist_kernel(const int32_t* __restrict__ idx, int* __restrict__ hist,
+                            int chunk_shift, int T, int K, int E, int* err) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * K) return;
+  int t = i / K, ex = idx[i];
+  if (ex < 0 || ex >= E) { set_device_error(err, MOE_DEVERR_INDEX); return; }
+  atomicAdd(&hist[(size_t)(t >> chunk_shift) * E + ex], 1);
+}
+
+// counts[e] = sum over chunks of hist[c][e]
+__global__ void counts_kernel(const int* __restrict__ hist, int n_chunks, int E, int* counts) {
+  int ex = blockIdx.x * blockDim.x + threadIdx.x;
+  if (ex >= E) return;
+  int run = 0;
+  for (int c = 0; c < n_chunks; ++c) run += hist[(size_t)c * E + ex];
+  counts[ex] = run;
+}
+
+// Exclusive scan of one value per thread over a block of up to 1024 threads.
+__device__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_sums[32];
+  const int lane = threadIdx.x % kWarp, warp = threadIdx.x / kWarp;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < kWarp; off <<= 1) {
+    int y = __shfl_up_sync(kFull, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == kWarp - 1) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int nw = (blockDim.x + kWarp - 1) / kWarp;
+    int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < kWarp; off <<= 1) {
+      int y = __shfl_up_sync(kFull, w, off);
+      if (lane >= off) w += y;
+    }
+    warp_sums[lane] = w;    // inclusive
+  }
+  __syncthreads();
+  int base = warp > 0 ? warp_sums[warp - 1] : 0;
+  int nw = (blockDim.x + kWarp - 1) / kWarp;
+  if (total) *total = warp_sums[nw - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// a4/a5 bookkeeping (one block of 1024 threads, E <= 1024):
+// counts, kept = min(counts, C), offsets = exclusive scan of kept, and the
+// per-chunk base rank chunk_base[c][e] = sum_{c' < c} hist[c'][e].
+__global__ void __launch_bounds__(1024)
+scan_kernel(const int* __restrict__ hist, int n_chunks, int E, int cap, int* __restrict__ counts,
+            int* __restrict__ kept, int* __restrict__ offsets, int* __restrict__ chunk_base) {
+  const int ex = threadIdx.x;
+  int kv = 0;
+  if (ex < E) {
+    int run = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      int v = hist[(size_t)c * E + ex];
+      chunk_base[(size_t)c * E + ex] = run;
+      run += v;
+    }
+    if (counts) counts[ex] = run;
+    kv = run < cap ? run : cap;
+    kept[ex] = kv;
+  }
+  int total;
+  int off = block_exclusive_scan(kv, &total);
+  if (ex < E) offsets[ex] = off;
+  if (ex == 0) offsets[E] = total;
+}
+
+// Group table of the grouped FFN: groups 0..E_r-1 are the routed experts
+// (rows offsets[g] .. offsets[g+1]-1), groups E_r..E_r+E_s-1 the shared experts
+// (T rows each, row base j*T); unit prefixes for the two GEMMs, with tiles of
+// bm rows and nt_* column tiles per group.
+__global__ void __launch_bounds__(1024)
+groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, int nt_gu_r,
+              int nt_gu_s, int nt_dn_r, int nt_dn_s, int* __restrict__ grp_rows,
+              int* __restrict__ grp_row0, int* __restrict__ pre_gu, int* __restrict__ pre_dn,
+              int max_rows, int* err) {
+  const int G = E_r + E_s;
+  // routed offsets must be non-decreasing within [0, max_rows]; otherwise no
+  // unit is scheduled (the FFN writes nothing) and the error word is set
+  int bad = 0;
+  for (int g = threadIdx.x; g < E_r; g += blockDim.x)
+    bad |= offsets[g + 1] < offsets[g];
+  if (threadIdx.x == 0) bad |= offsets[0] < 0 || offsets[E_r] > max_rows;
+  bad = __syncthreads_or(bad);
+  if (bad && threadIdx.x == 0) set_device_error(err, MOE_DEVERR_INDEX);
+  // G <= 1032: each thread handles up to two groups (g and g + 1024 folded)
+  int carry_gu = 0, carry_dn = 0;
+  for (int base = 0; base < G; base += blockDim.x) {
+    int g = base + threadIdx.x;
+    int rows = 0, row0 = 0, ugu = 0, udn = 0;
+    if (g < G) {
+      if (g < E_r) { row0 = offsets[g]; rows = bad ? 0 : offsets[g + 1] - row0; }
+      else { rows = bad ? 0 : T; row0 = (g - E_r) * T; }
+      int mt = (rows + bm - 1) / bm;
+      ugu = mt * (g < E_r ? nt_gu_r : nt_gu_s);
+      udn = mt * (g < E_r ? nt_dn_r : nt_dn_s);
+      grp_rows[g] = rows;
+      grp_row0[g] = row0;
+    }
+    int tot_gu, tot_dn;
+    int pgu = block_exclusive_scan(ugu, &tot_gu);
+    int pdn = block_exclusive_scan(udn, &tot_dn);
+    if (g < G) { pre_gu[g] = carry_gu + pgu; pre_dn[g] = carry_dn + pdn; }
+    carry_gu += tot_gu;
+    carry_dn += tot_dn;
+  }
+  if (threadIdx.x == 0) { pre_gu[G] = carry_gu; pre_dn[G] = carry_dn; }
+}
+
+// a5: stable scatter.  One block of 256 threads per chunk of 256 tokens; the
+// rank of (t, e) among the chunk's tokens choosing e comes from per-warp lane
+// masks, so rows stay in ascending token order within each expert.
+__global__ void __launch_bounds__(256)
+scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gates,
+               const int* __restrict__ offsets, const int* __restrict__ chunk_base, int cap,
+               int T, int K, int E, int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of,
+               float* __restrict__ row_gate, int* err) {
+  extern __shared__ uint32_t sm_scatter[];
+  uint32_t* wmask = sm_scatter;                        // [8][E]
+  int* wbase = reinterpret_cast<int*>(sm_scatter + 8 * E);   // [8][E]
+  const int chunk = blockIdx.x, tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+  for (int i = tid; i < 8 * E; i += blockDim.x) wmask[i] = 0;
+  __syncthreads();
+  const int t = chunk * 256 + tid;
+  const bool valid = t < T;
+  if (valid) {
+    for (int k = 0; k < K; ++k) {
+      int ex = idx[(size_t)t * K + k];
+      if (ex < 0 || ex >= E) { set_device_error(err, MOE_DEVERR_INDEX); continue; }
+      atomicOr(&wmask[warp * E + ex], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int ex = tid; ex < E; ex += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < 8; ++w) { wbase[w * E + ex] = run; run += __popc(wmask[w * E + ex]); }
+  }
+  __syncthreads();
+  if (valid) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      int ex = idx[(size_t)t * K + k];
+      int row = -1;
+      if (ex >= 0 && ex < E) {
+        int r = chunk_base[(size_t)chunk * E + ex] + wbase[warp * E + ex] +
+                __popc(wmask[warp * E + ex] & lt);
+        if (r < cap) {
+          row = offsets[ex] + r;
+          if (row >= offsets[ex + 1]) {           // self-check: rank past the expert's rows
+            set_device_error(err, MOE_DEVERR_INDEX);
+            row = -1;
+          } else {
+            perm_tok[row] = t;
+            if (row_gate) row_gate[row] = gates[(size_t)t * K + k];
+          }
+        }
+      }
+      row_of[(size_t)t * K + k] = row;
+    }
+  }
+}
+
+// x_perm[r] = h[perm_tok[r]] for r < offsets[E] (one warp per row, 16-byte moves)
+__global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* __restrict__ perm_tok,
+                                   const int* __restrict__ n_rows_ptr, uint4* __restrict__ x_perm,
+                                   int vec_per_row, int n_tok, int max_rows, int* err) {
+  const int n = min(*n_rows_ptr, max_rows);
+  const int lane = threadIdx.x % kWarp;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
+  const int nw = gridDim.x * blockDim.x / kWarp;
+  for (int r = gw; r < n; r += nw) {
+    const int t = perm_tok[r];
+    if ((unsigned)t >= (unsigned)n_tok) {            // self-check: never read outside h
+      if (lane == 0) set_device_error(err, MOE_DEVERR_INDEX);
+      continue;
+    }
+    const uint4* src = h + (size_t)t * vec_per_row;
+    uint4* dst = x_perm + (size_t)r * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += kWarp) dst[v] = src[v];
+  }
+}
+
+// a8: y_t = res*h_t + sum_j shared[j,t] + sum_k slot[row_of[t,k]], fp32 in that order.
+template <typename T>
+__global__ void __launch_bounds__(128)
+combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
+               const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int K,
+               int E_s, int add_residual, int n_slot_rows) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int t = blockIdx.x;
+  int rows[32];
+  for (int k = 0; k < K; ++k) {
+    int r = row_of[(size_t)t * K + k];
+    rows[k] = r < n_slot_rows ? r : -1;       // self-check: never read past the slot rows
+  }
+  for (int c = threadIdx.x * VEC; c < d; c += blockDim.x * VEC) {
+    float acc[VEC];
+    {
+      uint4 raw = *reinterpret_cast<const uint4*>(h + (size_t)t * d + c);
+      const T* v = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = add_residual ? to_f32(v[i]) : 0.f;
+    }
+    for (int j = 0; j < E_s; ++j) {
+      uint4 raw = *reinterpret_cast<const uint4*>(shared + ((size_t)j * n_tok + t) * d + c);
+      const T* v = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
+    }
+    for (int k = 0; k < K; ++k) {
+      if (rows[k] < 0) continue;
+      uint4 raw = *reinterpret_cast<const uint4*>(slot + (size_t)rows[k] * d + c);
+      const T* v = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
+    }
+    uint4 out;
+    T* o = reinterpret_cast<T*>(&out);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) o[i] = from_f32<T>(acc[i]);
+    *reinterpret_cast<uint4*>(y + (size_t)t * d + c) = out;
+  }
+}
+
+// a9: b_i += gamma * sign(K*T - E_r*c_i) (one fp32 add), and MaxVio.
+__global__ void __launch_bounds__(1024)
+bias_update_kernel(const int* __restrict__ counts, float* __restrict__ b, float gamma,
+                   float* __restrict__ max_vio, int E, int K, int T) {
+  __shared__ int smax[32];
+  const int ex = threadIdx.x;
+  int c = ex < E ? counts[ex] : 0;
+  if (ex < E && b) {
+    long long diff = (long long)K * T - (long long)E * c;
+    float step = diff > 0 ? gamma : (diff < 0 ? -gamma : 0.0f);
+    b[ex] = __fadd_rn(b[ex], step);
+  }
+  int m = c;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(kFull, m, off));
+  if (threadIdx.x % kWarp == 0) smax[threadIdx.x / kWarp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0 && max_vio) {
+    int mm = 0;
+    for (int w = 0; w < (int)(blockDim.x / kWarp); ++w) mm = max(mm, smax[w]);
+    double cbar = (double)K * (double)T / (double)E;
+    max_vio[0] = (float)(((double)mm - cbar) / cbar);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
+                          cudaStream_t st) {
+  dim3 grid((T + 63) / 64, (E + 63) / 64);
+  if (dtype == MOE_DTYPE_BF16)
+    router_logits_simt_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)h, e, z, T, d, E);
+  else
+    router_logits_simt_kernel<float><<<grid, 256, 0, st>>>((const float*)h, e, z, T, d, E);
+}
+
+void launch_select(const float* in, int in_is_scores, const float* bias, int score_fn,
+                   float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
+                   int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st) {
+  const int warps = 8;
+  dim3 grid((T + warps - 1) / warps);
+  int kpl = (E + 31) / 32;
+#define MOE_SEL(N) select_kernel<N><<<grid, warps * 32, 0, st>>>(in, in_is_scores, bias, score_fn, \
+      s_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
+  if (kpl <= 1) MOE_SEL(1);
+  else if (kpl <= 2) MOE_SEL(2);
+  else if (kpl <= 4) MOE_SEL(4);
+  else if (kpl <= 8) MOE_SEL(8);
+  else if (kpl <= 16) MOE_SEL(16);
+  else MOE_SEL(32);
+#undef MOE_SEL
+}
+
+void launch_hist(const int32_t* idx, int* hist, int chunk_shift, int T, int K, int E, int* err,
+                 cudaStream_t st) {
+  int n = T * K;
+  hist_kernel<<<(n + 255) / 256, 256, 0, st>>>(idx, hist, chunk_shift, T, K, E, err);
+}
+
+void launch_counts(const int* hist, int n_chunks, int E, int* counts, cudaStream_t st) {
+  counts_kernel<<<(E + 255) / 256, 256, 0, st>>>(hist, n_chunks, E, counts);
+}
+
+void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int* kept,
+                 int* offsets, int* chunk_base, cudaStream_t st) {
+  scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, cap, counts, kept, offsets, chunk_base);
+}
+
+void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
+                   int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
+                   int* pre_dn, int max_rows, int* err, cudaStream_t st) {
+  groups_kernel<<<1, 1024, 0, st>>>(offsets, E_r, E_s, T, bm, nt_gu_r, nt_gu_s, nt_dn_r, nt_dn_s,
+                                    grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err);
+}
+
+void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
+                    const int* chunk_base, int cap, int T, int K, int E, int32_t* perm_tok,
+                    int32_t* row_of, float* row_gate, int* err, cudaStream_t st) {
+  int n_chunks = (T + 255) / 256;
+  size_t smem = (size_t)16 * E * sizeof(uint32_t);
+  scatter_kernel<<<n_chunks, 256, smem, st>>>(idx, gates, offsets, chunk_base, cap, T, K, E,
+                                              perm_tok, row_of, row_gate, err);
+}
+
+void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
+                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st) {
+  int vec = d * elem_bytes / 16;
+  int warps = max_rows < 148 * 64 ? max_rows : 148 * 64;
+  if (warps < 1) warps = 1;
+  int blocks = (warps * 32 + 255) / 256;
+  gather_rows_kernel<<<blocks, 256, 0, st>>>((const uint4*)h, perm_tok, n_rows_ptr, (uint4*)x_perm,
+                                             vec, n_tok, max_rows, err);
+}
+
+void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
+                    void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
+                    int n_slot_rows, cudaStream_t st) {
+  if (dtype == MOE_DTYPE_BF16)
+    combine_kernel<bf16><<<T, 128, 0, st>>>((const bf16*)h, (const bf16*)slot, (const bf16*)shared,
+                                            row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
+  else
+    combine_kernel<float><<<T, 128, 0, st>>>((const float*)h, (const float*)slot,
+                                             (const float*)shared, row_of, (float*)y, T, d, K, E_s,
+                                             add_residual, n_slot_rows);
+}
+
+void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
+                        int T, cudaStream_t st) {
+  bias_update_kernel<<<1, 1024, 0, st>>>(counts, b, gamma, max_vio, E, K, T);
+}
+
+}  // namespace moe
