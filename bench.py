@@ -423,10 +423,16 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling only: run the workload with this many routed experts (smaller "
+                         "device footprint for ncu captures); not a bench configuration")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = mi.WORKLOADS[args.workload]
+    if args.experts:
+        w = w.with_(name=f"{w.name}_E{args.experts}", E_r=args.experts,
+                    n_groups=min(w.n_groups, args.experts // 4) if w.n_groups > 1 else 1)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -27,7 +27,9 @@
  *  - Pointers are DEVICE pointers unless stated otherwise; the caller owns
  *    every buffer (inputs, outputs and the workspace `ws`).  The library never
  *    allocates or frees device memory.  Arrays are dense, row-major, with no
- *    padding; every device pointer must be 16-byte aligned.
+ *    padding.  Activation and weight matrices (h, x, y, slot, shared_out, x_perm,
+ *    the expert weights) must be 16-byte aligned; every other array 4-byte
+ *    aligned; the workspace 256-byte aligned.
  *  - Activations and expert weights have the element type cfg->dtype
  *    (MOE_DTYPE_F32: float; MOE_DTYPE_BF16: bfloat16 bits in uint16).
  *    Centroids e, biases b, scores and gates are always float32; indices and

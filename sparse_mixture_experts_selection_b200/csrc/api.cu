@@ -133,6 +133,8 @@ moe_status cuda_status() {
 #define MOE_NONNULL(p) do { if (!(p)) return fail(MOE_ERR_INVALID_ARG, #p " is NULL"); \
     if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, #p " is not 16-byte aligned"); } while (0)
 #define MOE_ALIGNED(p) do { if ((p) && !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, #p " is not 16-byte aligned"); } while (0)
+#define MOE_ALIGNED4(p) do { if ((p) && (reinterpret_cast<uintptr_t>(p) & 3u)) return fail(MOE_ERR_INVALID_ARG, #p " is not 4-byte aligned"); } while (0)
+#define MOE_NONNULL4(p) do { if (!(p)) return fail(MOE_ERR_INVALID_ARG, #p " is NULL"); MOE_ALIGNED4(p); } while (0)
 
 template <typename T> T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -223,9 +225,9 @@ moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const
                      int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
-  if (!s_in) { MOE_NONNULL(h); MOE_NONNULL(e); }
-  MOE_ALIGNED(s_in); MOE_ALIGNED(s_out); MOE_ALIGNED(b); MOE_ALIGNED(counts);
-  MOE_NONNULL(idx); MOE_NONNULL(gates);
+  if (!s_in) { MOE_NONNULL(h); MOE_NONNULL4(e); }
+  MOE_ALIGNED4(s_in); MOE_ALIGNED4(s_out); MOE_ALIGNED4(b); MOE_ALIGNED4(counts);
+  MOE_NONNULL4(idx); MOE_NONNULL4(gates);
   const Layout L = make_layout(c);
   MOE_CHECK(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -246,8 +248,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* idx, const float* g
                        void* stream) {
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
-  MOE_NONNULL(idx); MOE_NONNULL(offsets); MOE_NONNULL(perm_tok); MOE_NONNULL(row_of); MOE_NONNULL(kept);
-  MOE_ALIGNED(gates); MOE_ALIGNED(h); MOE_ALIGNED(row_gate); MOE_ALIGNED(x_perm);
+  MOE_NONNULL4(idx); MOE_NONNULL4(offsets); MOE_NONNULL4(perm_tok); MOE_NONNULL4(row_of); MOE_NONNULL4(kept);
+  MOE_ALIGNED4(gates); MOE_ALIGNED(h); MOE_ALIGNED4(row_gate); MOE_ALIGNED(x_perm);
   if (row_gate && !gates) return fail(MOE_ERR_INVALID_ARG, "row_gate needs gates");
   if (x_perm && !h) return fail(MOE_ERR_INVALID_ARG, "x_perm needs h");
   const Layout L = make_layout(c);
@@ -276,8 +278,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ff
   MOE_CHECK(moe_expert_ffn_workspace_size(cfg, n_experts, d_ffn, max_rows, &need));
   const moe_config& c = *cfg;
   if (c.dtype == MOE_DTYPE_BF16 && d_ffn < 64) return fail(MOE_ERR_UNSUPPORTED, "bf16 needs d_ffn >= 64");
-  MOE_NONNULL(offsets); MOE_NONNULL(x); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down);
-  MOE_NONNULL(out); MOE_ALIGNED(row_scale);
+  MOE_NONNULL4(offsets); MOE_NONNULL(x); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down);
+  MOE_NONNULL(out); MOE_ALIGNED4(row_scale);
   MOE_CHECK(check_ws(ws, ws_bytes, need));
   if (max_rows == 0) return MOE_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -306,7 +308,7 @@ moe_status moe_combine(const moe_config* cfg, const void* h, const void* slot,
                        const void* shared_out, const int32_t* row_of, void* y, void* stream) {
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
-  MOE_NONNULL(h); MOE_NONNULL(slot); MOE_NONNULL(row_of); MOE_NONNULL(y);
+  MOE_NONNULL(h); MOE_NONNULL(slot); MOE_NONNULL4(row_of); MOE_NONNULL(y);
   if (c.E_s > 0) MOE_NONNULL(shared_out);
   moe::launch_combine(h, slot, shared_out, row_of, y, c.T, c.d_model, c.K, c.E_s, c.add_residual,
                       c.dtype, 0x7FFFFFFF, static_cast<cudaStream_t>(stream));
@@ -317,7 +319,7 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float g
                            float* max_vio, void* stream) {
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
-  MOE_NONNULL(counts); MOE_NONNULL(b);
+  MOE_NONNULL4(counts); MOE_NONNULL4(b); MOE_ALIGNED4(max_vio);
   if (!std::isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not finite");
   moe::launch_bias_update(counts, b, gamma, max_vio, c.E_r, c.K, c.T, static_cast<cudaStream_t>(stream));
   return cuda_status();
@@ -333,14 +335,14 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
   MOE_NONNULL(h); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down); MOE_NONNULL(y);
-  if (!s_in) MOE_NONNULL(e);
+  if (!s_in) MOE_NONNULL4(e);
   if (c.E_s > 0) { MOE_NONNULL(ws_gate); MOE_NONNULL(ws_up); MOE_NONNULL(ws_down); }
   if (update_bias) {
-    MOE_NONNULL(b);
+    MOE_NONNULL4(b);
     if (!std::isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not finite");
   }
-  MOE_ALIGNED(b); MOE_ALIGNED(s_in); MOE_ALIGNED(idx_out); MOE_ALIGNED(gates_out);
-  MOE_ALIGNED(counts_out); MOE_ALIGNED(kept_out); MOE_ALIGNED(s_out); MOE_ALIGNED(max_vio_out);
+  MOE_ALIGNED4(b); MOE_ALIGNED4(s_in); MOE_ALIGNED4(idx_out); MOE_ALIGNED4(gates_out);
+  MOE_ALIGNED4(counts_out); MOE_ALIGNED4(kept_out); MOE_ALIGNED4(s_out); MOE_ALIGNED4(max_vio_out);
   const Layout L = make_layout(c);
   MOE_CHECK(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
