@@ -221,6 +221,31 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
                              void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory for one (a caller whose device memory all belongs to its own pool, a
+ * caller enqueuing work while another thread captures a CUDA graph, a
+ * latency-critical caller that cannot accept cudaMalloc's implicit
+ * synchronisation).  The pages have no counterpart: this is a deployment
+ * variant of moe_permute with the same arguments, outputs and results,
+ * minus ws/ws_bytes.
+ *   dev_error: optional int32 DEVICE word that receives MOE_DEVERR_INDEX if an
+ *   expert index outside [0, E_r) is met (NULL: not reported).
+ * Scratch: a fixed 2 MiB + 64 KiB array in the library's own device memory,
+ * held on every GPU that loads the library until exit.  Shapes needing more
+ * (2 * ceil(T/256) * E_r + E_r + 64 int32 words) return MOE_ERR_UNSUPPORTED
+ * before anything is enqueued.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and must therefore come before
+ * any stream capture.  All calls share the array and it keeps the last call's
+ * contents (the call clears what must start at zero): calls whose work
+ * overlaps on the GPU, e.g. on two streams, race and must be serialised by the
+ * caller.  No cudaMalloc/cudaFree or allocating library routine is called.
+ */
+moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* idx, const float* gates,
+                               const void* h, int32_t* offsets, int32_t* perm_tok,
+                               int32_t* row_of, int32_t* kept, float* row_gate, void* x_perm,
+                               int32_t* dev_error, void* stream);
+
+/*
  * Profiling support.  When n_events > 0, every later moe_layer_forward call in
  * this thread records the caller's CUDA events (cudaEvent_t handles, created
  * and owned by the caller) on its stream at the phase boundaries:

@@ -69,6 +69,7 @@ SIGNATURES = {
     "moe_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_clear_device_error": (ctypes.c_int, [_P, _P]),
     "moe_set_phase_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), _I32]),
+    "moe_permute_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 # phases of moe_layer_forward marked by moe_set_phase_events (between marks i and i+1)
@@ -153,6 +154,15 @@ def moe_permute(cfg, idx, gates, h, offsets, perm_tok, row_of, kept, row_gate, x
     _check(lib().moe_permute(ctypes.byref(cfg), _ptr(idx), _ptr(gates), _ptr(h), _ptr(offsets),
                              _ptr(perm_tok), _ptr(row_of), _ptr(kept), _ptr(row_gate), _ptr(x_perm),
                              _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_permute_noalloc(cfg, idx, gates, h, offsets, perm_tok, row_of, kept, row_gate, x_perm,
+                        dev_error=None, stream=None):
+    """moe_permute with no workspace: for callers that cannot allocate device
+    memory (see include/moe.h); scratch is a fixed array inside the library."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _ptr(idx), _ptr(gates), _ptr(h), _ptr(offsets),
+                                     _ptr(perm_tok), _ptr(row_of), _ptr(kept), _ptr(row_gate),
+                                     _ptr(x_perm), _ptr(dev_error), _stream(stream)))
 
 
 def moe_expert_ffn(cfg, n_experts, d_ffn, max_rows, offsets, x, w_gate, w_up, w_down, row_scale,
