@@ -108,7 +108,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -243,6 +243,31 @@ def workload_config(w):
 
 
 # ---------------------------------------------------------------------------
+# replicas (N > 1): one process per GPU, no data-path collective
+# ---------------------------------------------------------------------------
+
+def h_stream_id(rank: int, step: int) -> int:
+    """Tensor id of the token batch of `step` on replica `rank` (distinct per rank)."""
+    return mi.h_tensor_id(rank * 100000 + step)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The max of a per-rank float over all ranks (timing only)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every replica's tokens over the slowest replica's time."""
+    return world * tokens_per_step * steps / (max_ms / 1000.0)
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -274,7 +299,7 @@ def run_ours(args, w, rank, world, local_rank):
     H = []
     for i in range(n_steps):
         t = torch.empty((w.T, w.d_model), dtype=dt, device=dev)
-        native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, mi.h_tensor_id(rank * 100000 + i), 0, 1.0,
+        native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, h_stream_id(rank, i), 0, 1.0,
                            stream=stream.cuda_stream)
         H.append(t)
     cfg = moe.config_for(w)
@@ -285,9 +310,10 @@ def run_ours(args, w, rank, world, local_rank):
     max_vio = torch.zeros(n_steps, dtype=torch.float32, device=dev)
     update = w.gamma > 0
 
-    def step(i, hh=None):
+    def step(i, hh=None, yy=None):
         moe.moe_layer_forward(cfg, H[i] if hh is None else hh, e, b, W["gate"], W["up"], W["down"],
-                              W["sgate"], W["sup"], W["sdown"], y, ws, counts_out=counts[i],
+                              W["sgate"], W["sup"], W["sdown"], y if yy is None else yy, ws,
+                              counts_out=counts[i],
                               kept_out=kept[i], update_bias=update, gamma=w.gamma,
                               max_vio_out=max_vio[i:i + 1])
 
@@ -318,11 +344,7 @@ def run_ours(args, w, rank, world, local_rank):
     moe.moe_set_phase_events([])
     if world > 1:
         dist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     err = moe.moe_get_device_error(ws)
     if err:
         raise RuntimeError(f"device error word {err} after the timed region")
@@ -330,35 +352,59 @@ def run_ours(args, w, rank, world, local_rank):
     phase_ms = np.array([[evs[i].elapsed_time(evs[i + 1]) for i in range(n_ph - 1)] for evs in ph_events])
     kept_h = kept.cpu().numpy()[args.warmup:]
     vio_h = max_vio.cpu().numpy()
-    value = world * w.T * args.steps / (elapsed_ms / 1000.0)
+    value = job_throughput(world, w.T, args.steps, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
+        # Public API end to end: pinned host h in, layer, y back to pinned host,
+        # every step.  Copies run on a second stream, double-buffered, so the
+        # H2D of step j+1 and the D2H of step j overlap the compute of the
+        # neighbouring steps; the timed region spans the first H2D to the last D2H.
         pin_h = [H[i].cpu().pin_memory() for i in range(args.warmup, n_steps)]
-        y_host = torch.empty((w.T, w.d_model), dtype=dt).pin_memory()
-        h_dev = torch.empty_like(H[0])
+        y_host = [torch.empty((w.T, w.d_model), dtype=dt).pin_memory() for _ in range(2)]
+        h_dev = [torch.empty_like(H[0]) for _ in range(2)]
+        y_dev = [y, torch.empty_like(y)]
         b.copy_(b_after_warmup)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        main, cs = torch.cuda.current_stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        h_ready = [ev() for _ in range(args.steps)]
+        done = [ev() for _ in range(args.steps)]
+        y_read = [ev() for _ in range(args.steps)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(main)
+        cs.wait_event(e0)
+        with torch.cuda.stream(cs):
+            h_dev[0].copy_(pin_h[0], non_blocking=True)
+            h_ready[0].record(cs)
         for j in range(args.steps):
-            h_dev.copy_(pin_h[j], non_blocking=True)
-            step(args.warmup + j, h_dev)
-            y_host.copy_(y, non_blocking=True)
-        e1.record()
+            buf = j % 2
+            main.wait_event(h_ready[j])
+            if j >= 2:
+                main.wait_event(y_read[j - 2])          # y_dev[buf] has been read back
+            step(args.warmup + j, h_dev[buf], y_dev[buf])
+            done[j].record(main)
+            with torch.cuda.stream(cs):
+                if j + 1 < args.steps:
+                    if j >= 1:
+                        cs.wait_event(done[j - 1])      # h_dev[(j+1)%2] no longer in use
+                    h_dev[(j + 1) % 2].copy_(pin_h[j + 1], non_blocking=True)
+                    h_ready[j + 1].record(cs)
+                cs.wait_event(done[j])
+                y_host[buf].copy_(y_dev[buf], non_blocking=True)
+                y_read[j].record(cs)
+        main.wait_event(y_read[args.steps - 1])
+        e1.record(main)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         es = 2 if bf16 else 4
-        e2e = {"value": world * w.T * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
-               "h2d_bytes_per_step": w.T * w.d_model * es, "d2h_bytes_per_step": w.T * w.d_model * es}
+        e2e = {"value": job_throughput(world, w.T, args.steps, e2e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": w.T * w.d_model * es, "d2h_bytes_per_step": w.T * w.d_model * es,
+               "copies": "pinned host, second stream, double-buffered"}
 
     if rank != 0:
         return
@@ -375,11 +421,15 @@ def run_ours(args, w, rank, world, local_rank):
     gu_flops = float(np.mean([x[0] for x in gu]))
     gu_s = float(np.mean(gu_ms)) / 1000.0
     achieved = gu_bytes / gu_s / 1e9
+    # DRAM traffic per launch: the ncu capture's traffic/algorithmic ratio
+    # (profiles/traffic.json) scaled to this launch's algorithmic bytes
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            traffic = json.load(f).get(w.name, {}).get("ffn_gate_up")
+            rec = json.load(f).get("ffn_gate_up")
+        if rec:
+            traffic = rec["ratio"] * gu_bytes
     layer = [layer_work(w, k) for k in kept_h]
     l_flops = float(np.mean([x[0] for x in layer]))
     l_bytes = float(np.mean([x[1] for x in layer]))
@@ -423,6 +473,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling only: tokens per step (with --experts)")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: run the workload with this many routed experts (smaller "
                          "device footprint for ncu captures); not a bench configuration")
@@ -433,6 +485,8 @@ def main():
     if args.experts:
         w = w.with_(name=f"{w.name}_E{args.experts}", E_r=args.experts,
                     n_groups=min(w.n_groups, args.experts // 4) if w.n_groups > 1 else 1)
+    if args.tokens:
+        w = w.with_(name=f"{w.name}_T{args.tokens}", T=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -38,7 +38,7 @@ int64_t capacity_rows(const moe_config& c) {
 
 struct Layout {
   size_t err, scores, hist, chunk_base, counts, kept, offsets, grp_rows, grp_row0, pre_gu, pre_dn;
-  size_t idx, gates, row_of, perm_tok, row_gate, maxvio, x_perm, act_r, act_s, slot_r, slot_s;
+  size_t idx, gates, row_of, perm_tok, row_gate, maxvio, x_perm, act_r, act_s, slot_r, slot_s, e3;
   size_t total;
   int n_chunks;
   int64_t cap, R;
@@ -55,7 +55,10 @@ Layout make_layout(const moe_config& c) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.err = take(kAlign);
-  L.scores = take((size_t)c.T * c.E_r * 4);
+  // fp32 logits: split-K partial sums of the tensor-core router (bf16 layers)
+  // or the CUDA-core logits (fp32 layers)
+  L.scores = take((size_t)(c.dtype == MOE_DTYPE_BF16 ? moe::kRouterMaxSplits : 1) * c.T * c.E_r * 4);
+  L.e3 = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)3 * c.E_r * c.d_model * 2 : 0);
   L.hist = take((size_t)L.n_chunks * c.E_r * 4);
   L.chunk_base = take((size_t)L.n_chunks * c.E_r * 4);
   L.counts = take((size_t)c.E_r * 4);
@@ -141,6 +144,30 @@ template <typename T> T* at(void* ws, size_t off) {
 }
 
 bool use_tensor_cores(int dtype) { return dtype == MOE_DTYPE_BF16; }
+
+// a1-a4: logits (tensor cores for bf16, CUDA cores for fp32) unless scores are
+// fed, then activation, selection, gates and the per-chunk histogram.
+moe_status run_route(const moe_config& c, const Layout& L, void* ws, const void* h, const float* e,
+                     const float* b, const float* s_in, float* s_out, int32_t* idx, float* gates,
+                     cudaStream_t st) {
+  int* hist = at<int>(ws, L.hist);
+  float* scores = at<float>(ws, L.scores);
+  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
+  int n_parts = 1;
+  if (!s_in) {
+    if (use_tensor_cores(c.dtype)) {
+      cudaError_t er = moe::launch_router_tc(h, e, at<void>(ws, L.e3), scores, c.T, c.d_model, c.E_r,
+                                             at<int>(ws, L.err), &n_parts, st);
+      if (er != cudaSuccess) return fail(MOE_ERR_CUDA, "tensor-core router launch: %s", cudaGetErrorString(er));
+    } else {
+      moe::launch_router_logits(h, c.dtype, e, scores, c.T, c.d_model, c.E_r, st);
+    }
+  }
+  moe::launch_select(s_in ? s_in : scores, n_parts, s_in != nullptr,
+                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
+                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
+  return cuda_status();
+}
 
 // Caller-provided CUDA events recorded at the phase boundaries of
 // moe_layer_forward (profiling support; see moe_set_phase_events).
@@ -231,14 +258,8 @@ moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const
   const Layout L = make_layout(c);
   MOE_CHECK(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int* hist = at<int>(ws, L.hist);
-  float* scores = at<float>(ws, L.scores);
-  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
-  if (!s_in) moe::launch_router_logits(h, c.dtype, e, scores, c.T, c.d_model, c.E_r, st);
-  moe::launch_select(s_in ? s_in : scores, s_in != nullptr,
-                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
-                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
-  if (counts) moe::launch_counts(hist, L.n_chunks, c.E_r, counts, st);
+  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, idx, gates, st));
+  if (counts) moe::launch_counts(at<int>(ws, L.hist), L.n_chunks, c.E_r, counts, st);
   return cuda_status();
 }
 
@@ -348,8 +369,6 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   int* err = at<int>(ws, L.err);
-  int* hist = at<int>(ws, L.hist);
-  float* scores = at<float>(ws, L.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   float* gates = gates_out ? gates_out : at<float>(ws, L.gates);
   int* counts = counts_out ? counts_out : at<int>(ws, L.counts);
@@ -362,14 +381,10 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
 
   // a1-a4: affinity, selection, gates, per-chunk histogram
   mark_phase(0, st);
-  cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
-  if (!s_in) moe::launch_router_logits(h, c.dtype, e, scores, c.T, c.d_model, c.E_r, st);
-  moe::launch_select(s_in ? s_in : scores, s_in != nullptr,
-                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
-                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
+  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, idx, gates, st));
   // a5: counts, capacity, offsets, stable scatter, row gather
   mark_phase(1, st);
-  moe::launch_scan(hist, L.n_chunks, c.E_r, (int)L.cap, counts, kept, offsets,
+  moe::launch_scan(at<int>(ws, L.hist), L.n_chunks, c.E_r, (int)L.cap, counts, kept, offsets,
                    at<int>(ws, L.chunk_base), st);
   moe::launch_scatter(idx, gates, offsets, at<int>(ws, L.chunk_base), (int)L.cap, c.T, c.K, c.E_r,
                       perm_tok, row_of, row_gate, err, st);

@@ -21,6 +21,7 @@
 // MMA issuer (one thread), warps 2..5 = epilogue (TMEM -> registers -> global).
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the
 // epilogue of one unit overlaps the MMAs of the next.
+#include <algorithm>
 #include <cuda.h>
 #include "common.cuh"
 #include "kernels.h"
@@ -41,7 +42,7 @@ constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
-enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
+enum { EPI_SWIGLU = 0, EPI_SCALE = 1, EPI_ROUTER = 2 };
 
 struct Params {
   CUtensorMap a_r, a_s;       // A: routed rows / shared rows
@@ -58,19 +59,54 @@ struct Params {
   uint16_t* out_s;
   const float* row_scale;     // routed rows' gates (EPI_SCALE), may be null
   int* err;
+  // EPI_ROUTER: z partial sums over split-K ranges of the virtual reduction
+  // [h | h | h] . [e_hi | e_mid | e_lo]^T (no group table)
+  int r_T, r_E, r_mtiles, r_ntiles, r_ks, r_nkd, r_per;
+  float* zpart;               // [r_ks, r_T, r_E]
 };
 
-__device__ __forceinline__ void decode(const Params& p, int u, int& g, int& mt, int& nt) {
-  int lo = 0, hi = p.G;
+// One work unit: group g (routed / shared), row tile, column tile and the
+// range of 64-wide k-blocks it reduces over.
+struct Unit {
+  int g, mt, nt, kb0, nk;
+  bool sh;
+};
+
+template <int EPI>
+__device__ __forceinline__ int total_units(const Params& p) {
+  if (EPI == EPI_ROUTER) return p.r_mtiles * p.r_ntiles * p.r_ks;
+  return __ldg(p.prefix + p.G);
+}
+
+template <int EPI>
+__device__ __forceinline__ Unit decode(const Params& p, int u) {
+  Unit w;
+  if (EPI == EPI_ROUTER) {
+    // row tile fastest: CTAs running together read the same centroid tiles
+    w.g = 0; w.sh = false;
+    w.mt = u % p.r_mtiles;
+    int rest = u / p.r_mtiles;
+    const int ks = rest % p.r_ks;
+    w.nt = rest / p.r_ks;
+    w.kb0 = ks * p.r_per;
+    w.nk = min(3 * p.r_nkd, w.kb0 + p.r_per) - w.kb0;
+    w.nt = w.nt * p.r_ks + ks;          // packed (column tile, split) for the epilogue
+    return w;
+  }
+  int lo = 0, hi = p.G;                  // prefix[lo] <= u < prefix[lo + 1]
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
     if (__ldg(p.prefix + mid) <= u) lo = mid; else hi = mid;
   }
-  g = lo;
-  int local = u - __ldg(p.prefix + g);
-  int mtiles = (__ldg(p.grp_rows + g) + BM - 1) / BM;
-  mt = local % mtiles;
-  nt = local / mtiles;
+  w.g = lo;
+  w.sh = lo >= p.E_r;
+  int local = u - __ldg(p.prefix + lo);
+  int mtiles = (__ldg(p.grp_rows + lo) + BM - 1) / BM;
+  w.mt = local % mtiles;
+  w.nt = local / mtiles;
+  w.kb0 = 0;
+  w.nk = ((w.sh ? p.k_s : p.k_r) + BK - 1) / BK;
+  return w;
 }
 
 // Wait without giving up on *abort (used to drain copies and MMAs in flight
@@ -87,6 +123,36 @@ __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __e
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Tensor-map coordinates of the A and B tiles of k-block i of unit w.
+template <int EPI>
+struct TileCoords {
+  const CUtensorMap *am, *b0, *b1;
+  int ax, ay, bx, by;
+};
+
+template <int EPI>
+__device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Unit& w, int i) {
+  TileCoords<EPI> c;
+  c.am = w.sh ? &p.a_s : &p.a_r;
+  c.b0 = w.sh ? &p.b0_s : &p.b0_r;
+  c.b1 = w.sh ? &p.b1_s : &p.b1_r;
+  int brow;
+  if (EPI == EPI_ROUTER) {
+    c.ay = w.mt * BM;
+    brow = (w.nt / p.r_ks) * BN;
+    const int part = (w.kb0 + i) / p.r_nkd;     // virtual k-block -> (centroid part, k)
+    c.ax = c.bx = ((w.kb0 + i) - part * p.r_nkd) * BK;
+    c.by = part * p.r_E + brow;
+  } else {
+    const int e = w.sh ? w.g - p.E_r : w.g;
+    c.ay = ((EPI == EPI_SWIGLU && w.sh) ? 0 : __ldg(p.grp_row0 + w.g)) + w.mt * BM;
+    brow = e * (w.sh ? p.wrows_s : p.wrows_r) + w.nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
+    c.ax = c.bx = (w.kb0 + i) * BK;
+    c.by = brow;
+  }
+  return c;
 }
 
 template <int EPI>
@@ -122,7 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = __ldg(p.prefix + p.G);
+  const int total = total_units<EPI>(p);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -131,26 +197,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       uint32_t phase = 0;
       int issued = 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
-        int g, mt, nt;
-        decode(p, u, g, mt, nt);
-        const bool sh = g >= p.E_r;
-        const int e = sh ? g - p.E_r : g;
-        const CUtensorMap* am = sh ? &p.a_s : &p.a_r;
-        const int arow = ((EPI == EPI_SWIGLU && sh) ? 0 : __ldg(p.grp_row0 + g)) + mt * BM;
-        const int wrows = sh ? p.wrows_s : p.wrows_r;
-        const int brow = e * wrows + nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
-        const CUtensorMap* b0 = sh ? &p.b0_s : &p.b0_r;
-        const CUtensorMap* b1 = sh ? &p.b1_s : &p.b1_r;
-        const int nk = ((sh ? p.k_s : p.k_r) + BK - 1) / BK;
-        for (int kb = 0; kb < nk; ++kb) {
+        const Unit w = decode<EPI>(p, u);
+        for (int i = 0; i < w.nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
+          const TileCoords<EPI> c = tile_coords<EPI>(p, w, i);
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, am, &full[stage], kb * BK, arow);
+          tma_load_2d(sA + stage * A_BYTES, c.am, &full[stage], c.ax, c.ay);
           if (EPI == EPI_SWIGLU) {
-            tma_load_2d(sB + stage * B_BYTES, b0, &full[stage], kb * BK, brow);
-            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, b1, &full[stage], kb * BK, brow);
+            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
+            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, c.b1, &full[stage], c.bx, c.by);
           } else {
-            tma_load_2d(sB + stage * B_BYTES, b0, &full[stage], kb * BK, brow);
+            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -171,15 +228,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
-        int g, mt, nt;
-        decode(p, u, g, mt, nt);
-        const bool sh = g >= p.E_r;
-        const int nk = ((sh ? p.k_s : p.k_r) + BK - 1) / BK;
+        const int nk = decode<EPI>(p, u).nk;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {      // kb counts this unit's k-blocks
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
@@ -207,19 +261,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      int g, mt, nt;
-      decode(p, u, g, mt, nt);
-      const bool sh = g >= p.E_r;
-      const int rows = __ldg(p.grp_rows + g);
+      const Unit w = decode<EPI>(p, u);
+      const int mt = w.mt, nt = w.nt;
+      const bool sh = w.sh;
+      const int rows = EPI == EPI_ROUTER ? p.r_T : __ldg(p.grp_rows + w.g);
       const int m = mt * BM + r;
       const bool valid = m < rows;
-      const size_t orow = (size_t)__ldg(p.grp_row0 + g) + m;
+      const size_t orow = (EPI == EPI_ROUTER ? 0 : (size_t)__ldg(p.grp_row0 + w.g)) + m;
       const int ncols = sh ? p.ncols_s : p.ncols_r;
       uint16_t* out = (sh ? p.out_s : p.out_r) + orow * ncols;
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == EPI_SWIGLU) {
+      if (EPI == EPI_ROUTER) {
+        // fp32 partial logits of split (nt % ks) for experts of column tile nt / ks
+        const int ks = nt % p.r_ks, ct = nt / p.r_ks;
+        float* zrow = p.zpart + ((size_t)ks * p.r_T + m) * p.r_E;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float dv[32];
+          tmem_ld32(tb + c, dv);
+          const int col0 = ct * BN + c;
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              if (col0 + 4 * v < p.r_E)
+                *reinterpret_cast<float4*>(zrow + col0 + 4 * v) =
+                    make_float4(dv[4 * v], dv[4 * v + 1], dv[4 * v + 2], dv[4 * v + 3]);
+          }
+        }
+      } else if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           float gv[32], uv[32];
@@ -320,6 +391,79 @@ static int num_sms() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 1;
+}
+
+// e (fp32) = e_hi + e_mid + e_lo exactly, each term bf16: e_hi = RN_bf16(e),
+// the residual e - e_hi is exact in fp32 (Sterbenz) and carries at most 16
+// significant bits, e_mid takes 8 of them and the last residual fits in bf16.
+__global__ void split_centroids_kernel(const float* __restrict__ e, __nv_bfloat16* __restrict__ e3,
+                                       size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float x = e[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const float r1 = __fsub_rn(x, __bfloat162float(hi));
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+    e3[i] = hi;
+    e3[n + i] = mid;
+    e3[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+// Split-K plan of the router GEMM: enough splits to fill the SMs, and never
+// more than kRouterMaxKbPerSplit k-blocks per split -- the tensor core's fp32
+// accumulation over long K drifts (observed 7e-6 in s at d = 7168 with 84
+// k-blocks per split), so long reductions are cut into short partial sums that
+// the select kernel adds in fp32, in split order.
+void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per) {
+  const int base = ((T + tc::BM - 1) / tc::BM) * ((E + tc::BN - 1) / tc::BN);
+  const int total = 3 * ((d + tc::BK - 1) / tc::BK);
+  int k0 = n_sms / base;
+  k0 = k0 < 1 ? 1 : k0;
+  int p = (total + k0 - 1) / k0;
+  if (p > kRouterMaxKbPerSplit) p = kRouterMaxKbPerSplit;
+  if ((total + p - 1) / p > kRouterMaxSplits) p = (total + kRouterMaxSplits - 1) / kRouterMaxSplits;
+  *per = p;
+  *ks = (total + p - 1) / p;           // every split non-empty
+}
+
+cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpart, int T, int d,
+                             int E, int* err, int* ks_out, cudaStream_t st) {
+  using namespace tc;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_ROUTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    attr_done[dev] = true;
+  }
+  const size_t n = (size_t)E * d;
+  split_centroids_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 148 * 8), 256, 0, st>>>(
+      e, reinterpret_cast<__nv_bfloat16*>(e3), n);
+  int ks, per;
+  router_split_plan(T, d, E, num_sms(), &ks, &per);
+  Params p{};
+  bool ok = true;
+  ok &= make_tmap(&p.a_r, h, (uint64_t)T, d, BM);
+  ok &= make_tmap(&p.a_s, h, (uint64_t)T, d, BM);
+  ok &= make_tmap(&p.b0_r, e3, (uint64_t)3 * E, d, BN);
+  ok &= make_tmap(&p.b1_r, e3, (uint64_t)3 * E, d, BN);
+  ok &= make_tmap(&p.b0_s, e3, (uint64_t)3 * E, d, BN);
+  ok &= make_tmap(&p.b1_s, e3, (uint64_t)3 * E, d, BN);
+  if (!ok) return cudaErrorInvalidValue;
+  p.r_T = T; p.r_E = E;
+  p.r_mtiles = (T + BM - 1) / BM;
+  p.r_ntiles = (E + BN - 1) / BN;
+  p.r_ks = ks; p.r_per = per;
+  p.r_nkd = (d + BK - 1) / BK;
+  p.zpart = zpart;
+  p.G = 1; p.E_r = 1;
+  p.err = err;
+  const int units = p.r_mtiles * p.r_ntiles * ks;
+  const int grid = std::min(units, num_sms());
+  grouped_gemm_kernel<EPI_ROUTER><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  *ks_out = ks;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {

@@ -21,7 +21,8 @@ struct FfnArgs {
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
                           cudaStream_t st);
-void launch_select(const float* in, int in_is_scores, const float* bias, int score_fn,
+// in: n_parts arrays [T, E] (logits partial sums, added in order) or the scores
+void launch_select(const float* in, int n_parts, int in_is_scores, const float* bias, int score_fn,
                    float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
                    int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st);
 void launch_hist(const int32_t* idx, int* hist, int chunk_shift, int T, int K, int E, int* err,
@@ -46,6 +47,15 @@ void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio
 int simt_bm();
 int simt_bn();
 void launch_ffn_simt(const FfnArgs& a, int which, cudaStream_t st);
+
+// Router logits on the tensor cores: split e into three bf16 terms (e3 =
+// [3, E, d] bf16 scratch) and write fp32 partial logits zpart [ks, T, E] over
+// ks split-K ranges (summed in order by the select kernel).
+constexpr int kRouterMaxSplits = 16;
+constexpr int kRouterMaxKbPerSplit = 24;
+void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per);
+cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpart, int T, int d,
+                             int E, int* err, int* ks_out, cudaStream_t st);
 
 int tc_bm();
 int tc_cols_gateup();

@@ -84,7 +84,7 @@ __device__ __forceinline__ void warp_best(float& k, int& i) {
 
 template <int KPL>
 __global__ void __launch_bounds__(256)
-select_kernel(const float* __restrict__ in, int in_is_scores, const float* __restrict__ bias,
+select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const float* __restrict__ bias,
               int score_fn, float* __restrict__ s_out, int32_t* __restrict__ idx,
               float* __restrict__ gates, int* __restrict__ hist, int chunk_shift, int T, int E,
               int K, int n_groups, int topk_groups, int group_topn) {
@@ -98,6 +98,9 @@ select_kernel(const float* __restrict__ in, int in_is_scores, const float* __res
   for (int j = 0; j < KPL; ++j) {
     int ex = j * kWarp + lane;
     s[j] = ex < E ? row[ex] : 0.f;
+    // logits from split-K partial sums: added in split order (deterministic)
+    for (int q = 1; q < n_parts; ++q)
+      if (ex < E) s[j] = __fadd_rn(s[j], row[(size_t)q * T * E + ex]);
   }
   if (!in_is_scores) {
     if (score_fn == MOE_SCORE_SIGMOID) {
@@ -142,24 +145,49 @@ select_kernel(const float* __restrict__ in, int in_is_scores, const float* __res
     if (j * kWarp + lane < E) eligible |= 1u << j;
   if (n_groups > 1 && group_topn > 0) {
     const int gsz = E / n_groups;
+    int grp[KPL];                                  // group of each held expert
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) grp[j] = (j * kWarp + lane) / gsz;
     float G[32];
     for (int g = 0; g < n_groups; ++g) {
-      uint32_t used = 0;
-      float acc = 0.f;
-      for (int r = 0; r < group_topn; ++r) {
-        float bk = -INFINITY;
-        int bi = 0x7FFFFFFF;
+      float acc;
+      if (group_topn == 2) {
+        // the two largest keys of the group by one pairwise warp reduction
+        // (their sum does not depend on how ties among them are ordered)
+        float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
         for (int j = 0; j < KPL; ++j) {
-          int ex = j * kWarp + lane;
-          if (ex < E && ex / gsz == g && !(used >> j & 1u) && beats(key[j], ex, bk, bi)) {
-            bk = key[j];
-            bi = ex;
+          if (j * kWarp + lane < E && grp[j] == g) {
+            const float v = key[j];
+            if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
           }
         }
-        warp_best(bk, bi);
-        if ((bi & (kWarp - 1)) == lane) used |= 1u << (bi / kWarp);
-        acc = r == 0 ? bk : __fadd_rn(acc, bk);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float o1 = __shfl_xor_sync(kFull, m1, off), o2 = __shfl_xor_sync(kFull, m2, off);
+          const float hi = fmaxf(m1, o1), lo = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+          m1 = hi; m2 = lo;
+        }
+        acc = __fadd_rn(m1, m2);
+      } else {
+        // general case: the group_topn largest keys in descending order
+        uint32_t used = 0;
+        acc = 0.f;
+        for (int r = 0; r < group_topn; ++r) {
+          float bk = -INFINITY;
+          int bi = 0x7FFFFFFF;
+#pragma unroll
+          for (int j = 0; j < KPL; ++j) {
+            int ex = j * kWarp + lane;
+            if (ex < E && grp[j] == g && !(used >> j & 1u) && beats(key[j], ex, bk, bi)) {
+              bk = key[j];
+              bi = ex;
+            }
+          }
+          warp_best(bk, bi);
+          if ((bi & (kWarp - 1)) == lane) used |= 1u << (bi / kWarp);
+          acc = r == 0 ? bk : __fadd_rn(acc, bk);
+        }
       }
       G[g] = acc;
     }
@@ -172,8 +200,7 @@ select_kernel(const float* __restrict__ in, int in_is_scores, const float* __res
     }
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
-      int ex = j * kWarp + lane;
-      if (ex < E && !(keep >> (ex / gsz) & 1u)) eligible &= ~(1u << j);
+      if (j * kWarp + lane < E && !(keep >> grp[j] & 1u)) eligible &= ~(1u << j);
     }
   }
 
@@ -410,7 +437,13 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* _
     }
     const uint4* src = h + (size_t)t * vec_per_row;
     uint4* dst = x_perm + (size_t)r * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += kWarp) dst[v] = src[v];
+    // 4 independent 16-byte loads in flight per lane before the stores
+    int v = lane;
+    for (; v + 3 * kWarp < vec_per_row; v += 4 * kWarp) {
+      const uint4 a = src[v], b = src[v + kWarp], c = src[v + 2 * kWarp], e = src[v + 3 * kWarp];
+      dst[v] = a; dst[v + kWarp] = b; dst[v + 2 * kWarp] = c; dst[v + 3 * kWarp] = e;
+    }
+    for (; v < vec_per_row; v += kWarp) dst[v] = src[v];
   }
 }
 
@@ -493,13 +526,13 @@ void launch_router_logits(const void* h, int dtype, const float* e, float* z, in
     router_logits_simt_kernel<float><<<grid, 256, 0, st>>>((const float*)h, e, z, T, d, E);
 }
 
-void launch_select(const float* in, int in_is_scores, const float* bias, int score_fn,
+void launch_select(const float* in, int n_parts, int in_is_scores, const float* bias, int score_fn,
                    float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
                    int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st) {
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps);
   int kpl = (E + 31) / 32;
-#define MOE_SEL(N) select_kernel<N><<<grid, warps * 32, 0, st>>>(in, in_is_scores, bias, score_fn, \
+#define MOE_SEL(N) select_kernel<N><<<grid, warps * 32, 0, st>>>(in, n_parts, in_is_scores, bias, score_fn, \
       s_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
   if (kpl <= 1) MOE_SEL(1);
   else if (kpl <= 2) MOE_SEL(2);
@@ -536,7 +569,14 @@ void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
                     const int* chunk_base, int cap, int T, int K, int E, int32_t* perm_tok,
                     int32_t* row_of, float* row_gate, int* err, cudaStream_t st) {
   int n_chunks = (T + 255) / 256;
-  size_t smem = (size_t)16 * E * sizeof(uint32_t);
+  size_t smem = (size_t)16 * E * sizeof(uint32_t);      // 64 KB at E = 1024
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 16 * 1024 * 4);
+    attr_done[dev] = true;
+  }
   scatter_kernel<<<n_chunks, 256, smem, st>>>(idx, gates, offsets, chunk_base, cap, T, K, E,
                                               perm_tok, row_of, row_gate, err);
 }

@@ -139,7 +139,11 @@ def check_close(y_gpu: np.ndarray, y_ref: np.ndarray, h: np.ndarray, tol: float,
     err = float(np.max(diff))
     r_y = rms(y_ref)
     r_d = rms(y_ref - (np.asarray(h, np.float64) if residual else 0.0))
-    assert err <= tol * r_y, (err, r_y)
+    if residual:
+        # BASELINE's bar (its workloads all carry the residual); without the
+        # residual y is the bf16-rounded expert sum itself and only the
+        # rounding-aware check below applies
+        assert err <= tol * r_y, (err, r_y)
     strict = float(np.max(diff - out_eps * np.abs(y_ref)))
     assert strict <= tol * r_d, (strict, r_d)
     return err, r_y, r_d
