@@ -95,7 +95,10 @@ def down_work(w, kept: np.ndarray):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi samples every 20 ms from construction on (nvidia-smi needs
+    ~0.1 s to start, longer than a timed region); summary() keeps only the
+    samples whose timestamps fall inside the window passed to mark()."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
@@ -103,8 +106,7 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.lines = []
-
-    def __enter__(self):
+        self.window = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
@@ -114,13 +116,15 @@ class ClockSampler:
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
-        return self
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def __exit__(self, *exc):
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    def stop(self):
         if self.proc:
             self.proc.terminate()
             try:
@@ -129,21 +133,28 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        import datetime
         rows = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != 7:
+            if len(parts) != 8:
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
             except ValueError:
                 continue
-        if not rows:
-            return None
+        if self.window:
+            lo, hi = self.window
+            inside = [r for r in rows if lo <= r[0] <= hi]
+        else:
+            inside = rows
+        if not inside:
+            return {"samples": 0, "note": "no nvidia-smi sample fell inside the timed region"}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for _, _, _, r in inside for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
 
 
 # ---------------------------------------------------------------------------
@@ -317,6 +328,7 @@ def run_ours(args, w, rank, world, local_rank):
                               kept_out=kept[i], update_bias=update, gamma=w.gamma,
                               max_vio_out=max_vio[i:i + 1])
 
+    clocks = ClockSampler(torch.cuda.current_device())
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -334,13 +346,14 @@ def run_ours(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clocks:
-        t_start.record()
-        for j in range(args.steps):
-            moe.moe_set_phase_events(ph_events[j])
-            step(args.warmup + j)
-        t_end.record()
-        torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record()
+    for j in range(args.steps):
+        moe.moe_set_phase_events(ph_events[j])
+        step(args.warmup + j)
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks.mark(wall0, time.time())
     moe.moe_set_phase_events([])
     if world > 1:
         dist.barrier()
@@ -406,6 +419,7 @@ def run_ours(args, w, rank, world, local_rank):
                "h2d_bytes_per_step": w.T * w.d_model * es, "d2h_bytes_per_step": w.T * w.d_model * es,
                "copies": "pinned host, second stream, double-buffered"}
 
+    clocks.stop()
     if rank != 0:
         return
 
@@ -455,7 +469,9 @@ def run_ours(args, w, rank, world, local_rank):
         "max_vio": [round(float(v), 4) for v in vio_h[args.warmup:]],
         "e2e": e2e,
         "clocks": clocks.summary(),
-        "gpu_launches": 10 * args.steps,
+        # our kernels per step: [centroid split + router GEMM | CUDA-core logits], select,
+        # scan, scatter, gather, group tables, gate/up GEMM, down GEMM, combine, bias step
+        "gpu_launches": (11 if bf16 else 10) * args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)

@@ -111,8 +111,9 @@ const char* moe_last_error_detail(void);
  * Required workspace bytes for moe_layer_forward with this config (an upper
  * bound for every other entry point with the same config).  *bytes is a HOST
  * pointer.  The workspace must be 256-byte aligned device memory; its first
- * 256 bytes hold the device error word, which the caller must zero once
- * (cudaMemset) before first use.
+ * 256 bytes are the library's control block (the device error word and the
+ * GEMM unit counters), which the caller must zero once (cudaMemset) before
+ * first use.
  */
 moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes);
 
@@ -124,6 +125,8 @@ moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes);
  *   s_in   [T, E_r] float32 scores to route from ("fed" mode: skips the affinity),
  *                   or NULL to compute s from h and e (fp32 logits).
  *   s_out  [T, E_r] float32: the scores used, or NULL.
+ *   z_out  [T, E_r] float32: the fp32 logits h_t . e_i, or NULL (not written
+ *                   in fed mode, when there are no logits).
  *   idx    [T, K]   int32 out: I_t in ascending expert index.
  *   gates  [T, K]   float32 out: g_{t,i} in the same order.
  *   counts [E_r]    int32 out: c_i (before any capacity drop), or NULL.
@@ -132,7 +135,7 @@ moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes);
  * Balancing -- DeepSeek-V3", How it works / Official code.
  */
 moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const float* b,
-                     const float* s_in, float* s_out, int32_t* idx, float* gates,
+                     const float* s_in, float* s_out, float* z_out, int32_t* idx, float* gates,
                      int32_t* counts, void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -207,6 +210,7 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float g
  *   ws_gate/ws_up [E_s, f_s, d], ws_down [E_s, d, f_s] (NULL when E_s = 0).
  *   y [T, d] out.  Optional outputs (NULL to skip): idx_out [T, K],
  *   gates_out [T, K], counts_out [E_r], kept_out [E_r], s_out [T, E_r],
+ *   z_out [T, E_r] (fp32 logits; not written in fed mode),
  *   max_vio_out (device float32 scalar; written whenever non-NULL).
  *   s_in: optional fed scores [T, E_r] (skips the affinity; e may then be NULL).
  * With update_bias, the routing of THIS call uses the incoming b and the step
@@ -216,9 +220,37 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
                              const void* w_gate, const void* w_up, const void* w_down,
                              const void* ws_gate, const void* ws_up, const void* ws_down,
                              const float* s_in, void* y, int32_t* idx_out, float* gates_out,
-                             int32_t* counts_out, int32_t* kept_out, float* s_out,
+                             int32_t* counts_out, int32_t* kept_out, float* s_out, float* z_out,
                              int32_t update_bias, float gamma, float* max_vio_out,
                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Router losses and logging over one batch (training-time reductions over the
+ * routing results; none of them changes the forward output):
+ *   stats[0] Switch auxiliary loss  alpha_aux * sum_i f_i P_i,
+ *            f_i = E_r/(K T) c_i, P_i = mean_t s'_{t,i}, s' = s / sum_j s_j
+ *            ("Sparse Mixture-of-Experts ...", section 1 equation; for softmax
+ *            routing s' = p);
+ *   stats[1] router z-loss  c_z / T * sum_t (logsumexp_i z_{t,i})^2 (same
+ *            section), 0 when z is NULL;
+ *   stats[2] sequence-wise balance loss ("Load Balancing -- DeepSeek-V3", How
+ *            it works): alpha_seq * sum_i f_i P_i within each sequence of
+ *            seq_len tokens (f_i normalised by K*seq_len), averaged over the
+ *            T/seq_len sequences; 0 when seq_len = 0;
+ *   stats[3] entropy of the load shares c_i / (K T) ("GPUs, memory and
+ *            failures", log_router);
+ *   stats[4] MaxVio;  stats[5] dropped rate 1 - sum kept / (K T) (0 when kept
+ *            is NULL).
+ *   s [T, E_r] scores and z [T, E_r] logits (NULL allowed) as exported by
+ *   moe_route / moe_layer_forward; idx [T, K]; kept [E_r] or NULL;
+ *   stats: 6 float32 on the device.  seq_len must be 0 or divide T.
+ *   ws: at least moe_router_stats_workspace_size bytes (its first 256 bytes
+ *   are not used by this call).  Deterministic (no floating-point atomics).
+ */
+moe_status moe_router_stats_workspace_size(const moe_config* cfg, int32_t seq_len, size_t* bytes);
+moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* z, const int32_t* idx,
+                            const int32_t* kept, int32_t seq_len, float alpha_aux, float c_z,
+                            float alpha_seq, float* stats, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_permute without a workspace, for callers that cannot allocate device
@@ -262,6 +294,17 @@ moe_status moe_set_phase_events(void* const* events, int32_t n_events);
  * pointer.  Returns MOE_ERR_DEVICE when the word is non-zero, MOE_OK otherwise.
  */
 moe_status moe_get_device_error(const void* ws, int32_t* code);
+
+/*
+ * Failure-detection self-test.  Enqueues one kernel whose only thread waits,
+ * through the same bounded shared-memory-barrier wait every GEMM pipeline
+ * stage uses, on a barrier that nothing ever arrives on.  After limit_ns
+ * (1 ms .. 2 s) the wait gives up, writes MOE_DEVERR_WAIT_TIMEOUT into the
+ * error word of ws (the first 256 bytes of a workspace) and the kernel
+ * returns: no trap, no hang, the context stays usable.  Read the word with
+ * moe_get_device_error after synchronising the stream.
+ */
+moe_status moe_selftest_bounded_wait(void* ws, int64_t limit_ns, void* stream);
 
 /* Zero the device error word of a workspace (enqueued on stream). */
 moe_status moe_clear_device_error(void* ws, void* stream);

@@ -332,3 +332,60 @@ def near_tie_tokens(s32: np.ndarray, b32: np.ndarray, K: int, n_groups: int = 1,
         nxt = srt[:, K]
         fragile |= np.isfinite(nxt) & ((srt[:, K - 1] - nxt) < gap)
     return fragile
+
+
+# ---------------------------------------------------------------------------
+# Router losses and logging ([SMoE] section 1 "Switch Auxiliary Loss & ST-MoE
+# Router z-Loss" equations; [DS3LB] "How it works", sequence-wise L_Bal;
+# [GMF] the bias card's log_router: MaxVio, dropped rate, router entropy)
+# ---------------------------------------------------------------------------
+
+def normalized_scores(s32: np.ndarray) -> np.ndarray:
+    """s'_{t,i} = s_{t,i} / sum_j s_{t,j} over all experts (equals p for softmax)."""
+    s = np.asarray(s32, np.float64)
+    return s / s.sum(axis=1, keepdims=True)
+
+
+def aux_loss(s32: np.ndarray, idx: np.ndarray, E_r: int, K: int, alpha: float) -> float:
+    """Switch auxiliary loss alpha * sum_i f_i P_i, f_i = E_r/(K T) * c_i,
+    P_i = mean_t s'_{t,i}."""
+    T = idx.shape[0]
+    f = E_r / (K * T) * load_counts(idx, E_r).astype(np.float64)
+    P = normalized_scores(s32).mean(axis=0)
+    return float(alpha * np.sum(f * P))
+
+
+def z_loss(z32: np.ndarray, c_z: float) -> float:
+    """Router z-loss c_z / T * sum_t (log sum_i exp z_{t,i})^2."""
+    z = np.asarray(z32, np.float64)
+    m = z.max(axis=1, keepdims=True)
+    lse = (m + np.log(np.exp(z - m).sum(axis=1, keepdims=True)))[:, 0]
+    return float(c_z * np.mean(lse ** 2))
+
+
+def seq_balance_loss(s32: np.ndarray, idx: np.ndarray, E_r: int, K: int, seq_len: int,
+                     alpha: float) -> float:
+    """Sequence-wise balance loss, averaged over the T/seq_len sequences:
+    alpha * sum_i f_i P_i per sequence, with f_i = E_r/(K S) * (selections of i
+    in the sequence) and P_i = mean over the sequence of s'_{t,i}."""
+    T = idx.shape[0]
+    sp = normalized_scores(s32)
+    total = 0.0
+    n_seq = T // seq_len
+    for b in range(n_seq):
+        rows = slice(b * seq_len, (b + 1) * seq_len)
+        f = E_r / (K * seq_len) * load_counts(idx[rows], E_r).astype(np.float64)
+        P = sp[rows].mean(axis=0)
+        total += alpha * np.sum(f * P)
+    return float(total / n_seq)
+
+
+def load_entropy(counts: np.ndarray) -> float:
+    """Entropy of the load shares, -sum share * log(max(share, 1e-9))."""
+    share = np.asarray(counts, np.float64) / np.sum(counts)
+    return float(-np.sum(share * np.log(np.maximum(share, 1e-9))))
+
+
+def dropped_rate(kept: np.ndarray, counts: np.ndarray) -> float:
+    """Fraction of (token, expert) pairs dropped by capacity, 1 - kept/selected."""
+    return float(1.0 - np.sum(kept) / np.sum(counts))

@@ -21,6 +21,8 @@ __all__ = [
     "MoeConfig", "MoeError", "lib", "config_for", "moe_workspace_size", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_expert_ffn_workspace_size", "moe_combine", "moe_bias_update",
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
+    "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
+    "moe_set_phase_events", "moe_selftest_bounded_wait",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
 
@@ -57,19 +59,23 @@ SIGNATURES = {
     "moe_last_error_detail": (ctypes.c_char_p, []),
     "moe_workspace_size": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_expert_ffn_workspace_size": (ctypes.c_int, [_P, _I32, _I32, _I32, ctypes.POINTER(ctypes.c_size_t)]),
-    "moe_route": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_route": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
     "moe_combine": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_P, _P, ctypes.c_float, _P, _P, _P]),
     "moe_layer_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
-                                         _P, _P, _P, _I32, ctypes.c_float, _P, _P, ctypes.c_size_t,
-                                         _P]),
+                                         _P, _P, _P, _P, _I32, ctypes.c_float, _P, _P,
+                                         ctypes.c_size_t, _P]),
+    "moe_router_stats_workspace_size": (ctypes.c_int, [_P, _I32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_router_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
+                                        ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "moe_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_clear_device_error": (ctypes.c_int, [_P, _P]),
     "moe_set_phase_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), _I32]),
     "moe_permute_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [_P, ctypes.c_int64, _P]),
 }
 
 # phases of moe_layer_forward marked by moe_set_phase_events (between marks i and i+1)
@@ -145,9 +151,27 @@ def alloc_workspace(nbytes: int, device="cuda"):
     return ws
 
 
-def moe_route(cfg, h, e, b, s_in, s_out, idx, gates, counts, ws, stream=None):
+def moe_route(cfg, h, e, b, s_in, s_out, idx, gates, counts, ws, stream=None, z_out=None):
     _check(lib().moe_route(ctypes.byref(cfg), _ptr(h), _ptr(e), _ptr(b), _ptr(s_in), _ptr(s_out),
-                           _ptr(idx), _ptr(gates), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)))
+                           _ptr(z_out), _ptr(idx), _ptr(gates), _ptr(counts), _ptr(ws), ws.numel(),
+                           _stream(stream)))
+
+
+def moe_router_stats_workspace_size(cfg: MoeConfig, seq_len: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_router_stats_workspace_size(ctypes.byref(cfg), int(seq_len), ctypes.byref(n)))
+    return n.value
+
+
+# order of the values moe_router_stats writes
+ROUTER_STATS = ["aux_loss", "z_loss", "seq_balance_loss", "load_entropy", "max_vio", "dropped_rate"]
+
+
+def moe_router_stats(cfg, s, z, idx, kept, stats, ws, seq_len=0, alpha_aux=0.01, c_z=1e-3,
+                     alpha_seq=1e-4, stream=None):
+    _check(lib().moe_router_stats(ctypes.byref(cfg), _ptr(s), _ptr(z), _ptr(idx), _ptr(kept),
+                                  int(seq_len), float(alpha_aux), float(c_z), float(alpha_seq),
+                                  _ptr(stats), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_permute(cfg, idx, gates, h, offsets, perm_tok, row_of, kept, row_gate, x_perm, ws, stream=None):
@@ -184,11 +208,12 @@ def moe_bias_update(cfg, counts, gamma, b, max_vio, stream=None):
 
 def moe_layer_forward(cfg, h, e, b, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, ws, *,
                       s_in=None, idx_out=None, gates_out=None, counts_out=None, kept_out=None,
-                      s_out=None, update_bias=False, gamma=0.0, max_vio_out=None, stream=None):
+                      s_out=None, z_out=None, update_bias=False, gamma=0.0, max_vio_out=None,
+                      stream=None):
     _check(lib().moe_layer_forward(
         ctypes.byref(cfg), _ptr(h), _ptr(e), _ptr(b), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(s_in), _ptr(y), _ptr(idx_out), _ptr(gates_out),
-        _ptr(counts_out), _ptr(kept_out), _ptr(s_out), int(bool(update_bias)), float(gamma),
+        _ptr(counts_out), _ptr(kept_out), _ptr(s_out), _ptr(z_out), int(bool(update_bias)), float(gamma),
         _ptr(max_vio_out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
@@ -205,6 +230,11 @@ def moe_set_phase_events(events) -> None:
     every later moe_layer_forward call in this thread; [] turns it off."""
     arr = (ctypes.c_void_p * max(1, len(events)))(*[ev.cuda_event for ev in events])
     _check(lib().moe_set_phase_events(arr, len(events)))
+
+
+def moe_selftest_bounded_wait(ws, limit_ns: int = 50_000_000, stream=None) -> None:
+    """Enqueue the failure-detection self-test (see include/moe.h)."""
+    _check(lib().moe_selftest_bounded_wait(_ptr(ws), int(limit_ns), _stream(stream)))
 
 
 def moe_clear_device_error(ws, stream=None) -> None:

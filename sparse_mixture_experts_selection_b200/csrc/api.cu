@@ -148,8 +148,8 @@ bool use_tensor_cores(int dtype) { return dtype == MOE_DTYPE_BF16; }
 // a1-a4: logits (tensor cores for bf16, CUDA cores for fp32) unless scores are
 // fed, then activation, selection, gates and the per-chunk histogram.
 moe_status run_route(const moe_config& c, const Layout& L, void* ws, const void* h, const float* e,
-                     const float* b, const float* s_in, float* s_out, int32_t* idx, float* gates,
-                     cudaStream_t st) {
+                     const float* b, const float* s_in, float* s_out, float* z_out, int32_t* idx,
+                     float* gates, cudaStream_t st) {
   int* hist = at<int>(ws, L.hist);
   float* scores = at<float>(ws, L.scores);
   cudaMemsetAsync(hist, 0, (size_t)L.n_chunks * c.E_r * 4, st);
@@ -164,8 +164,9 @@ moe_status run_route(const moe_config& c, const Layout& L, void* ws, const void*
     }
   }
   moe::launch_select(s_in ? s_in : scores, n_parts, s_in != nullptr,
-                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out, idx, gates,
-                     hist, kChunkShift, c.T, c.E_r, c.K, c.n_groups, c.topk_groups, c.group_topn, st);
+                     c.score_fn == MOE_SCORE_SIGMOID ? b : nullptr, c.score_fn, s_out,
+                     s_in ? nullptr : z_out, idx, gates, hist, kChunkShift, c.T, c.E_r, c.K,
+                     c.n_groups, c.topk_groups, c.group_topn, st);
   return cuda_status();
 }
 
@@ -190,7 +191,7 @@ moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int
                      a.E_s ? (a.f_s + bn_gu - 1) / bn_gu : 0, (a.d + bn_dn - 1) / bn_dn,
                      (a.d + bn_dn - 1) / bn_dn, const_cast<int*>(a.grp_rows),
                      const_cast<int*>(a.grp_row0), const_cast<int*>(a.pre_gu),
-                     const_cast<int*>(a.pre_dn), max_rows, a.err, st);
+                     const_cast<int*>(a.pre_dn), max_rows, a.err, a.tile_counters, st);
   if (phase_base >= 0) mark_phase(phase_base, st);
   for (int which = 0; which < 2; ++which) {
     if (tc) {
@@ -248,17 +249,17 @@ moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_expert
 }
 
 moe_status moe_route(const moe_config* cfg, const void* h, const float* e, const float* b,
-                     const float* s_in, float* s_out, int32_t* idx, float* gates,
+                     const float* s_in, float* s_out, float* z_out, int32_t* idx, float* gates,
                      int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
   MOE_CHECK(validate(cfg));
   const moe_config& c = *cfg;
   if (!s_in) { MOE_NONNULL(h); MOE_NONNULL4(e); }
-  MOE_ALIGNED4(s_in); MOE_ALIGNED4(s_out); MOE_ALIGNED4(b); MOE_ALIGNED4(counts);
+  MOE_ALIGNED4(s_in); MOE_ALIGNED4(s_out); MOE_ALIGNED4(z_out); MOE_ALIGNED4(b); MOE_ALIGNED4(counts);
   MOE_NONNULL4(idx); MOE_NONNULL4(gates);
   const Layout L = make_layout(c);
   MOE_CHECK(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, idx, gates, st));
+  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, z_out, idx, gates, st));
   if (counts) moe::launch_counts(at<int>(ws, L.hist), L.n_chunks, c.E_r, counts, st);
   return cuda_status();
 }
@@ -322,6 +323,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ff
   a.act_r = at<void>(ws, o); a.act_s = a.act_r;
   a.out_r = out; a.out_s = out;
   a.err = at<int>(ws, 0);
+  a.tile_counters = at<int>(ws, 64);   // spare words of the error block
   return run_ffn(c, a, offsets, max_rows, st);
 }
 
@@ -350,7 +352,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
                              const void* w_gate, const void* w_up, const void* w_down,
                              const void* ws_gate, const void* ws_up, const void* ws_down,
                              const float* s_in, void* y, int32_t* idx_out, float* gates_out,
-                             int32_t* counts_out, int32_t* kept_out, float* s_out,
+                             int32_t* counts_out, int32_t* kept_out, float* s_out, float* z_out,
                              int32_t update_bias, float gamma, float* max_vio_out,
                              void* ws, size_t ws_bytes, void* stream) {
   MOE_CHECK(validate(cfg));
@@ -363,7 +365,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
     if (!std::isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is not finite");
   }
   MOE_ALIGNED4(b); MOE_ALIGNED4(s_in); MOE_ALIGNED4(idx_out); MOE_ALIGNED4(gates_out);
-  MOE_ALIGNED4(counts_out); MOE_ALIGNED4(kept_out); MOE_ALIGNED4(s_out); MOE_ALIGNED4(max_vio_out);
+  MOE_ALIGNED4(counts_out); MOE_ALIGNED4(kept_out); MOE_ALIGNED4(s_out); MOE_ALIGNED4(z_out);
+  MOE_ALIGNED4(max_vio_out);
   const Layout L = make_layout(c);
   MOE_CHECK(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -381,7 +384,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
 
   // a1-a4: affinity, selection, gates, per-chunk histogram
   mark_phase(0, st);
-  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, idx, gates, st));
+  MOE_CHECK(run_route(c, L, ws, h, e, b, s_in, s_out, z_out, idx, gates, st));
   // a5: counts, capacity, offsets, stable scatter, row gather
   mark_phase(1, st);
   moe::launch_scan(at<int>(ws, L.hist), L.n_chunks, c.E_r, (int)L.cap, counts, kept, offsets,
@@ -405,6 +408,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   a.act_r = at<void>(ws, L.act_r); a.act_s = c.E_s ? at<void>(ws, L.act_s) : a.act_r;
   a.out_r = at<void>(ws, L.slot_r); a.out_s = c.E_s ? at<void>(ws, L.slot_s) : a.out_r;
   a.err = err;
+  a.tile_counters = err + 16;          // spare words of the error block
   MOE_CHECK(run_ffn(c, a, offsets, (int)L.R, st, 3));
   mark_phase(5, st);
   // a8: fixed-order combine with the residual
@@ -432,6 +436,54 @@ moe_status moe_get_device_error(const void* ws, int32_t* code) {
   if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_status();
   *code = v;
   return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+static size_t router_stats_bytes(const moe_config& c, int32_t seq_len) {
+  const int S = seq_len > 0 ? seq_len : c.T;
+  const size_t n_seq = (size_t)c.T / S;
+  const size_t n_ch = ((size_t)S + moe::kStatsChunk - 1) / moe::kStatsChunk;
+  return align_up(kAlign + align_up((size_t)c.T * 4) * 2 + align_up(n_seq * c.E_r * 4) +
+                  align_up(n_seq * n_ch * c.E_r * 4));
+}
+
+moe_status moe_router_stats_workspace_size(const moe_config* cfg, int32_t seq_len, size_t* bytes) {
+  MOE_CHECK(validate(cfg));
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  if (seq_len < 0 || (seq_len > 0 && cfg->T % seq_len))
+    return fail(MOE_ERR_INVALID_ARG, "seq_len=%d must be 0 or divide T=%d", seq_len, cfg->T);
+  *bytes = router_stats_bytes(*cfg, seq_len);
+  return MOE_OK;
+}
+
+moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* z, const int32_t* idx,
+                            const int32_t* kept, int32_t seq_len, float alpha_aux, float c_z,
+                            float alpha_seq, float* stats, void* ws, size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  MOE_CHECK(moe_router_stats_workspace_size(cfg, seq_len, &need));
+  const moe_config& c = *cfg;
+  MOE_NONNULL4(s); MOE_NONNULL4(idx); MOE_NONNULL4(stats); MOE_ALIGNED4(z); MOE_ALIGNED4(kept);
+  if (!std::isfinite(alpha_aux) || !std::isfinite(c_z) || !std::isfinite(alpha_seq))
+    return fail(MOE_ERR_INVALID_ARG, "non-finite loss coefficient");
+  MOE_CHECK(check_ws(ws, ws_bytes, need));
+  const int S = seq_len > 0 ? seq_len : c.T;
+  const size_t n_seq = (size_t)c.T / S;
+  size_t o = kAlign;
+  float* rowsum = at<float>(ws, o); o += align_up((size_t)c.T * 4);
+  float* lse2 = at<float>(ws, o); o += align_up((size_t)c.T * 4);
+  int* seq_counts = at<int>(ws, o); o += align_up(n_seq * c.E_r * 4);
+  float* pchunk = at<float>(ws, o);
+  moe::launch_router_stats(s, z, idx, kept, c.T, c.E_r, c.K, S, seq_len > 0, alpha_aux, c_z,
+                           alpha_seq, rowsum, lse2, seq_counts, pchunk, stats,
+                           static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
+moe_status moe_selftest_bounded_wait(void* ws, int64_t limit_ns, void* stream) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "ws is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(MOE_ERR_WORKSPACE, "ws is not 256-byte aligned");
+  if (limit_ns < 1000000 || limit_ns > 2000000000) return fail(MOE_ERR_INVALID_ARG, "limit_ns outside [1 ms, 2 s]");
+  moe::launch_bounded_wait_selftest((uint64_t)limit_ns, at<int>(ws, 0), static_cast<cudaStream_t>(stream));
+  return cuda_status();
 }
 
 moe_status moe_clear_device_error(void* ws, void* stream) {

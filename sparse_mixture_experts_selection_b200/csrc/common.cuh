@@ -84,14 +84,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 // set by another warp or when the time limit passes; in the latter case it
 // records MOE_DEVERR_WAIT_TIMEOUT and sets *abort so the other roles leave too.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
+                                          int* err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         set_device_error(err, MOE_DEVERR_WAIT_TIMEOUT);
         *abort = 1;
         return false;

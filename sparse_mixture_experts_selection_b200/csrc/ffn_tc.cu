@@ -39,7 +39,7 @@ constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1, EPI_ROUTER = 2 };
@@ -63,7 +63,12 @@ struct Params {
   // [h | h | h] . [e_hi | e_mid | e_lo]^T (no group table)
   int r_T, r_E, r_mtiles, r_ntiles, r_ks, r_nkd, r_per;
   float* zpart;               // [r_ks, r_T, r_E]
+  // dynamic schedule: units are claimed from this zeroed counter (null: static
+  // round-robin over the CTAs)
+  int* tile_counter;
 };
+
+constexpr int UNIT_RING = 4;     // units handed from the producer to the MMA / epilogue warps
 
 // One work unit: group g (routed / shared), row tile, column tile and the
 // range of 64-wide k-blocks it reduces over.
@@ -166,13 +171,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* unit_full = drain + 1;
+  uint64_t* unit_empty = unit_full + UNIT_RING;
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(unit_empty + UNIT_RING);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UNIT_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4 * kWarp); }
+    for (int s = 0; s < UNIT_RING; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1 + 4 * kWarp); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -196,7 +205,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      int slot = 0;
+      uint32_t uphase = 0;
+      for (int k = 0;; ++k) {
+        // claim the next unit and hand it to the MMA and epilogue warps (-1 = done)
+        int u = p.tile_counter ? atomicAdd(p.tile_counter, 1) : (int)blockIdx.x + k * (int)gridDim.x;
+        if (u >= total) u = -1;
+        if (!mbar_wait(&unit_empty[slot], uphase ^ 1u, abort_flag, p.err)) goto producer_done;
+        unit_ring[slot] = u;
+        mbar_arrive(&unit_full[slot]);
+        if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+        if (u < 0) break;
         const Unit w = decode<EPI>(p, u);
         for (int i = 0; i < w.nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
@@ -227,7 +246,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      int slot = 0;
+      uint32_t uphase = 0;
+      for (;;) {
+        if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
+        const int u = unit_ring[slot];
+        mbar_arrive(&unit_empty[slot]);
+        if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+        if (u < 0) break;
         const int nk = decode<EPI>(p, u).nk;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
@@ -260,7 +286,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     const int r = sub * 32 + lane;         // row within the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    int slot = 0;
+    uint32_t uphase = 0;
+    for (;;) {
+      if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
+      const int u = unit_ring[slot];
+      mbar_arrive(&unit_empty[slot]);
+      if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+      if (u < 0) break;
       const Unit w = decode<EPI>(p, u);
       const int mt = w.mt, nt = w.nt;
       const bool sh = w.sh;
@@ -518,6 +551,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
     p.row_scale = a.row_scale;
   }
   if (!ok) return cudaErrorInvalidValue;
+  p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
   const int grid = num_sms();
   if (which == 0)
     grouped_gemm_kernel<EPI_SWIGLU><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);

@@ -17,14 +17,15 @@ struct FfnArgs {
   const float* row_scale;
   void *act_r, *act_s, *out_r, *out_s;
   int* err;
+  int* tile_counters;   // [2] unit counters of the two GEMMs, zeroed by groups_kernel
 };
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
                           cudaStream_t st);
 // in: n_parts arrays [T, E] (logits partial sums, added in order) or the scores
 void launch_select(const float* in, int n_parts, int in_is_scores, const float* bias, int score_fn,
-                   float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
-                   int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st);
+                   float* s_out, float* z_out, int32_t* idx, float* gates, int* hist, int chunk_shift,
+                   int T, int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st);
 void launch_hist(const int32_t* idx, int* hist, int chunk_shift, int T, int K, int E, int* err,
                  cudaStream_t st);
 void launch_counts(const int* hist, int n_chunks, int E, int* counts, cudaStream_t st);
@@ -32,7 +33,7 @@ void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int
                  int* offsets, int* chunk_base, cudaStream_t st);
 void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
                    int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
-                   int* pre_dn, int max_rows, int* err, cudaStream_t st);
+                   int* pre_dn, int max_rows, int* err, int* tile_counters, cudaStream_t st);
 void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
                     const int* chunk_base, int cap, int T, int K, int E, int32_t* perm_tok,
                     int32_t* row_of, float* row_gate, int* err, cudaStream_t st);
@@ -43,6 +44,13 @@ void launch_combine(const void* h, const void* slot, const void* shared, const i
                     int n_slot_rows, cudaStream_t st);
 void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
                         int T, cudaStream_t st);
+void launch_bounded_wait_selftest(uint64_t limit_ns, int* err, cudaStream_t st);
+// Tokens per partial sum of the per-sequence score means (router statistics).
+constexpr int kStatsChunk = 64;
+void launch_router_stats(const float* s, const float* z, const int32_t* idx, const int32_t* kept,
+                         int T, int E, int K, int seq_len, int use_seq, float alpha_aux, float c_z,
+                         float alpha_seq, float* rowsum, float* lse2, int* seq_counts, float* pseq,
+                         float* stats, cudaStream_t st);
 
 int simt_bm();
 int simt_bn();

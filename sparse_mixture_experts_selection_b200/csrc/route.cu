@@ -85,7 +85,7 @@ __device__ __forceinline__ void warp_best(float& k, int& i) {
 template <int KPL>
 __global__ void __launch_bounds__(256)
 select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const float* __restrict__ bias,
-              int score_fn, float* __restrict__ s_out, int32_t* __restrict__ idx,
+              int score_fn, float* __restrict__ s_out, float* __restrict__ z_out, int32_t* __restrict__ idx,
               float* __restrict__ gates, int* __restrict__ hist, int chunk_shift, int T, int E,
               int K, int n_groups, int topk_groups, int group_topn) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
@@ -103,6 +103,11 @@ select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const
       if (ex < E) s[j] = __fadd_rn(s[j], row[(size_t)q * T * E + ex]);
   }
   if (!in_is_scores) {
+    if (z_out) {
+#pragma unroll
+      for (int j = 0; j < KPL; ++j)
+        if (j * kWarp + lane < E) z_out[(size_t)t * E + j * kWarp + lane] = s[j];
+    }
     if (score_fn == MOE_SCORE_SIGMOID) {
 #pragma unroll
       for (int j = 0; j < KPL; ++j) s[j] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-s[j])));
@@ -334,7 +339,8 @@ __global__ void __launch_bounds__(1024)
 groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, int nt_gu_r,
               int nt_gu_s, int nt_dn_r, int nt_dn_s, int* __restrict__ grp_rows,
               int* __restrict__ grp_row0, int* __restrict__ pre_gu, int* __restrict__ pre_dn,
-              int max_rows, int* err) {
+              int max_rows, int* err, int* tile_counters) {
+  if (tile_counters && threadIdx.x < 2) tile_counters[threadIdx.x] = 0;   // GEMM unit counters
   const int G = E_r + E_s;
   // routed offsets must be non-decreasing within [0, max_rows]; otherwise no
   // unit is scheduled (the FFN writes nothing) and the error word is set
@@ -460,7 +466,8 @@ combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __r
     int r = row_of[(size_t)t * K + k];
     rows[k] = r < n_slot_rows ? r : -1;       // self-check: never read past the slot rows
   }
-  for (int c = threadIdx.x * VEC; c < d; c += blockDim.x * VEC) {
+  // blockIdx.y splits a token's row over several blocks when there are few tokens
+  for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * VEC; c < d; c += blockDim.x * gridDim.y * VEC) {
     float acc[VEC];
     {
       uint4 raw = *reinterpret_cast<const uint4*>(h + (size_t)t * d + c);
@@ -515,8 +522,157 @@ bias_update_kernel(const int* __restrict__ counts, float* __restrict__ b, float 
 }
 
 // ---------------------------------------------------------------------------
+// Router losses and logging: Switch aux loss, router z-loss, sequence-wise
+// balance loss, load entropy, MaxVio, dropped rate.  Deterministic: integer
+// atomics only, every float sum in a fixed order.
+// ---------------------------------------------------------------------------
+
+// Per token: row sum of s (for s' = s / sum s), (logsumexp z)^2, and the
+// per-sequence selection counts.
+__global__ void __launch_bounds__(256)
+stats_token_kernel(const float* __restrict__ s, const float* __restrict__ z,
+                   const int32_t* __restrict__ idx, float* __restrict__ rowsum,
+                   float* __restrict__ lse2, int* __restrict__ seq_counts, int T, int E, int K,
+                   int seq_len) {
+  const int lane = threadIdx.x % kWarp;
+  const int t = blockIdx.x * (blockDim.x / kWarp) + threadIdx.x / kWarp;
+  if (t >= T) return;
+  float acc = 0.f;
+  for (int i = lane; i < E; i += kWarp) acc = __fadd_rn(acc, s[(size_t)t * E + i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, off));
+  if (z) {
+    float m = -INFINITY;
+    for (int i = lane; i < E; i += kWarp) m = fmaxf(m, z[(size_t)t * E + i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    float e = 0.f;
+    for (int i = lane; i < E; i += kWarp) e = __fadd_rn(e, expf(z[(size_t)t * E + i] - m));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) e = __fadd_rn(e, __shfl_xor_sync(kFull, e, off));
+    if (lane == 0) {
+      const float lse = m + logf(e);
+      lse2[t] = lse * lse;
+    }
+  }
+  if (lane == 0) rowsum[t] = acc;
+  if (lane < K) {
+    const int ex = idx[(size_t)t * K + lane];
+    if (ex >= 0 && ex < E) atomicAdd(&seq_counts[(size_t)(t / seq_len) * E + ex], 1);
+  }
+}
+
+// Per (sequence b, chunk j of kStatsChunk tokens, expert i): the partial sum
+// of s'_{t,i} over the chunk, so that a long sequence is spread over many
+// blocks; the final kernel adds the chunks of a sequence in ascending order.
+__global__ void __launch_bounds__(256)
+stats_seq_kernel(const float* __restrict__ s, const float* __restrict__ rowsum,
+                 float* __restrict__ pchunk, int E, int seq_len, int n_ch) {
+  const int b = blockIdx.x / n_ch, j = blockIdx.x % n_ch;
+  const int i = blockIdx.y * blockDim.x + threadIdx.x;
+  if (i >= E) return;
+  const size_t t0 = (size_t)b * seq_len + (size_t)j * kStatsChunk;
+  const int n = min(kStatsChunk, seq_len - j * kStatsChunk);
+  float acc = 0.f;
+  for (int t = 0; t < n; ++t) acc = __fadd_rn(acc, __fdiv_rn(s[(t0 + t) * E + i], rowsum[t0 + t]));
+  pchunk[(size_t)blockIdx.x * E + i] = acc;
+}
+
+// Block-wide sum of one value per thread in a fixed tree order.
+__device__ double block_sum_fixed(double v) {
+  __shared__ double part[32];
+  const int lane = threadIdx.x % kWarp, warp = threadIdx.x / kWarp;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  if (lane == 0) part[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < (int)(blockDim.x / kWarp); ++w) r += part[w];
+  __syncthreads();
+  return r;     // valid in thread 0
+}
+
+// Final reductions (one block of 1024 threads, one expert per thread).
+__global__ void __launch_bounds__(1024)
+stats_final_kernel(const float* __restrict__ pchunk, const int* __restrict__ seq_counts,
+                   const float* __restrict__ lse2, const int32_t* __restrict__ kept, int T, int E,
+                   int K, int seq_len, int n_ch, int use_seq, float alpha_aux, float c_z,
+                   float alpha_seq, float* __restrict__ stats) {
+  const int i = threadIdx.x;
+  const int n_seq = T / seq_len;
+  double c_i = 0.0, P_i = 0.0, seq_i = 0.0;
+  if (i < E) {
+    for (int b = 0; b < n_seq; ++b) {
+      const double cb = seq_counts[(size_t)b * E + i];
+      double pb = 0.0;
+      for (int j = 0; j < n_ch; ++j) pb += pchunk[((size_t)b * n_ch + j) * E + i];
+      pb /= seq_len;
+      c_i += cb;
+      P_i += pb;
+      seq_i += (double)E / ((double)K * seq_len) * cb * pb;
+    }
+    P_i /= n_seq;
+  }
+  const double f_i = (double)E / ((double)K * T) * c_i;
+  const double aux = block_sum_fixed(i < E ? f_i * P_i : 0.0);
+  const double seq = block_sum_fixed(i < E ? seq_i : 0.0);
+  const double share = c_i / ((double)K * T);
+  const double ent = block_sum_fixed((i < E && share > 0.0) ? -share * log(fmax(share, 1e-9)) : 0.0);
+  const double ksum = block_sum_fixed((i < E && kept) ? (double)kept[i] : 0.0);
+  __shared__ int cmax_s;
+  if (threadIdx.x == 0) cmax_s = 0;
+  __syncthreads();
+  if (i < E) atomicMax(&cmax_s, (int)c_i);
+  double zsum = 0.0;
+  for (int t = threadIdx.x; t < T && lse2; t += blockDim.x) zsum += lse2[t];
+  const double zl = block_sum_fixed(zsum);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double cbar = (double)K * T / E;
+    stats[0] = (float)(alpha_aux * aux);
+    stats[1] = lse2 ? (float)(c_z * zl / T) : 0.0f;
+    stats[2] = use_seq ? (float)(alpha_seq * seq / n_seq) : 0.0f;
+    stats[3] = (float)ent;
+    stats[4] = (float)(((double)cmax_s - cbar) / cbar);
+    stats[5] = kept ? (float)(1.0 - ksum / ((double)K * T)) : 0.0f;
+  }
+}
+
+// Failure-detection self-test: one thread waits, through the same bounded
+// mbarrier wait the GEMM pipelines use, on a barrier nothing arrives on.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait(&bar, 0, &abort_flag, err, limit_ns);     // never completes: times out
+}
+
+// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
+
+void launch_router_stats(const float* s, const float* z, const int32_t* idx, const int32_t* kept,
+                         int T, int E, int K, int seq_len, int use_seq, float alpha_aux, float c_z,
+                         float alpha_seq, float* rowsum, float* lse2, int* seq_counts, float* pchunk,
+                         float* stats, cudaStream_t st) {
+  const int n_seq = T / seq_len;
+  const int n_ch = (seq_len + kStatsChunk - 1) / kStatsChunk;
+  cudaMemsetAsync(seq_counts, 0, (size_t)n_seq * E * sizeof(int), st);
+  stats_token_kernel<<<(T + 7) / 8, 256, 0, st>>>(s, z, idx, rowsum, z ? lse2 : nullptr, seq_counts,
+                                                  T, E, K, seq_len);
+  stats_seq_kernel<<<dim3(n_seq * n_ch, (E + 255) / 256), 256, 0, st>>>(s, rowsum, pchunk, E, seq_len,
+                                                                       n_ch);
+  stats_final_kernel<<<1, 1024, 0, st>>>(pchunk, seq_counts, z ? lse2 : nullptr, kept, T, E, K,
+                                         seq_len, n_ch, use_seq, alpha_aux, c_z, alpha_seq, stats);
+}
+
+void launch_bounded_wait_selftest(uint64_t limit_ns, int* err, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, err);
+}
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
                           cudaStream_t st) {
   dim3 grid((T + 63) / 64, (E + 63) / 64);
@@ -527,13 +683,13 @@ void launch_router_logits(const void* h, int dtype, const float* e, float* z, in
 }
 
 void launch_select(const float* in, int n_parts, int in_is_scores, const float* bias, int score_fn,
-                   float* s_out, int32_t* idx, float* gates, int* hist, int chunk_shift, int T,
-                   int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st) {
+                   float* s_out, float* z_out, int32_t* idx, float* gates, int* hist, int chunk_shift,
+                   int T, int E, int K, int n_groups, int topk_groups, int group_topn, cudaStream_t st) {
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps);
   int kpl = (E + 31) / 32;
 #define MOE_SEL(N) select_kernel<N><<<grid, warps * 32, 0, st>>>(in, n_parts, in_is_scores, bias, score_fn, \
-      s_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
+      s_out, z_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
   if (kpl <= 1) MOE_SEL(1);
   else if (kpl <= 2) MOE_SEL(2);
   else if (kpl <= 4) MOE_SEL(4);
@@ -560,9 +716,9 @@ void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int
 
 void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
                    int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
-                   int* pre_dn, int max_rows, int* err, cudaStream_t st) {
+                   int* pre_dn, int max_rows, int* err, int* tile_counters, cudaStream_t st) {
   groups_kernel<<<1, 1024, 0, st>>>(offsets, E_r, E_s, T, bm, nt_gu_r, nt_gu_s, nt_dn_r, nt_dn_s,
-                                    grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err);
+                                    grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err, tile_counters);
 }
 
 void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
@@ -594,11 +750,17 @@ void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
                     void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
                     int n_slot_rows, cudaStream_t st) {
+  // enough blocks to fill the GPU even for decode-sized batches
+  const int nvec = d * (dtype == MOE_DTYPE_BF16 ? 2 : 4) / 16;
+  int split = (2 * 148 + T - 1) / T;
+  const int max_split = (nvec + 127) / 128;
+  split = split < 1 ? 1 : (split > max_split ? max_split : split);
+  const dim3 grid(T, split);
   if (dtype == MOE_DTYPE_BF16)
-    combine_kernel<bf16><<<T, 128, 0, st>>>((const bf16*)h, (const bf16*)slot, (const bf16*)shared,
+    combine_kernel<bf16><<<grid, 128, 0, st>>>((const bf16*)h, (const bf16*)slot, (const bf16*)shared,
                                             row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
   else
-    combine_kernel<float><<<T, 128, 0, st>>>((const float*)h, (const float*)slot,
+    combine_kernel<float><<<grid, 128, 0, st>>>((const float*)h, (const float*)slot,
                                              (const float*)shared, row_of, (float*)y, T, d, K, E_s,
                                              add_residual, n_slot_rows);
 }

@@ -103,6 +103,7 @@ class Layer:
         self.counts = torch.empty(E, dtype=torch.int32, device="cuda")
         self.kept = torch.empty(E, dtype=torch.int32, device="cuda")
         self.s = torch.empty((T, E), dtype=torch.float32, device="cuda")
+        self.z = torch.empty((T, E), dtype=torch.float32, device="cuda")
         self.max_vio = torch.empty(1, dtype=torch.float32, device="cuda")
 
     def forward(self, h, e, b, s_in=None, update_bias=False, gamma=0.0):
@@ -110,7 +111,7 @@ class Layer:
         moe.moe_layer_forward(self.cfg, h, e, b, W["gate"], W["up"], W["down"], W["sgate"], W["sup"],
                               W["sdown"], self.y, self.ws, s_in=s_in, idx_out=self.idx,
                               gates_out=self.gates, counts_out=self.counts, kept_out=self.kept,
-                              s_out=self.s, update_bias=update_bias, gamma=gamma,
+                              s_out=self.s, z_out=self.z, update_bias=update_bias, gamma=gamma,
                               max_vio_out=self.max_vio)
         return self.y
 
@@ -140,7 +141,7 @@ def check_close(y_gpu: np.ndarray, y_ref: np.ndarray, h: np.ndarray, tol: float,
     r_y = rms(y_ref)
     r_d = rms(y_ref - (np.asarray(h, np.float64) if residual else 0.0))
     if residual:
-        # BASELINE's bar (its workloads all carry the residual); without the
+        # the layer-output bar (stated for layers with the residual); without the
         # residual y is the bf16-rounded expert sum itself and only the
         # rounding-aware check below applies
         assert err <= tol * r_y, (err, r_y)

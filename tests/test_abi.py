@@ -91,27 +91,27 @@ def test_entry_points_validate_pointers_before_any_launch():
     P = FAKE
     # NULL inputs
     assert L.moe_layer_forward(ctypes.byref(c), None, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 0, 0.0, None, P, need, None) == 1
+                               None, None, None, None, None, None, 0, 0.0, None, P, need, None) == 1
     # too small / misaligned workspace
     assert L.moe_layer_forward(ctypes.byref(c), P, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 0, 0.0, None, P, need - 1, None) == 3
+                               None, None, None, None, None, None, 0, 0.0, None, P, need - 1, None) == 3
     assert L.moe_layer_forward(ctypes.byref(c), P, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 0, 0.0, None, P + 16, need, None) == 3
+                               None, None, None, None, None, None, 0, 0.0, None, P + 16, need, None) == 3
     # misaligned activation pointer
     assert L.moe_layer_forward(ctypes.byref(c), P + 4, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 0, 0.0, None, P, need, None) == 1
+                               None, None, None, None, None, None, 0, 0.0, None, P, need, None) == 1
     # update_bias without b, non-finite gamma
     assert L.moe_layer_forward(ctypes.byref(c), P, P, None, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 1, 0.1, None, P, need, None) == 1
+                               None, None, None, None, None, None, 1, 0.1, None, P, need, None) == 1
     assert L.moe_layer_forward(ctypes.byref(c), P, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 1, float("nan"), None, P, need, None) == 1
+                               None, None, None, None, None, None, 1, float("nan"), None, P, need, None) == 1
     # shared experts configured but their weights missing
     c2 = cfg_of("finegrained_64x1408")
     n2 = moe.moe_workspace_size(c2)
     assert L.moe_layer_forward(ctypes.byref(c2), P, P, P, P, P, P, None, None, None, None, P,
-                               None, None, None, None, None, 0, 0.0, None, P, n2, None) == 1
+                               None, None, None, None, None, None, 0, 0.0, None, P, n2, None) == 1
     # route: idx/gates required; permute: row_gate needs gates
-    assert L.moe_route(ctypes.byref(c), P, P, None, None, None, None, P, None, P, need, None) == 1
+    assert L.moe_route(ctypes.byref(c), P, P, None, None, None, None, None, P, None, P, need, None) == 1
     assert L.moe_permute(ctypes.byref(c), P, None, None, P, P, P, P, P, None, P, need, None) == 1
     assert L.moe_bias_update(ctypes.byref(c), None, 0.1, P, None, None) == 1
     assert L.moe_combine(ctypes.byref(c), P, None, None, P, P, None) == 1
@@ -122,3 +122,9 @@ def test_entry_points_validate_pointers_before_any_launch():
     assert L.moe_expert_ffn_workspace_size(ctypes.byref(c), 8, 128, 10, ctypes.byref(n)) == 0
     assert L.moe_expert_ffn(ctypes.byref(c), 8, 128, 10, P, P, P, P, P, None, P, P, n.value - 1, None) == 3
     assert L.moe_get_device_error(None, None) == 1
+    # router statistics: seq_len must divide T; stats required
+    n = ctypes.c_size_t(0)
+    assert L.moe_router_stats_workspace_size(ctypes.byref(c), 7, ctypes.byref(n)) == 1
+    assert L.moe_router_stats_workspace_size(ctypes.byref(c), 128, ctypes.byref(n)) == 0
+    assert L.moe_router_stats(ctypes.byref(c), P, None, P, None, 128, 0.01, 1e-3, 1e-4, None, P,
+                              n.value, None) == 1

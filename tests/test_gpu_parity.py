@@ -398,3 +398,17 @@ def test_layer_edge_cases(name):
     if name == "hot_expert_3_row_tiles":
         assert ref["kept"].max() > 2 * 128
     check_close(y.float().cpu().numpy(), ref["y"], h, tol_of(w), bool(w.add_residual), out_eps_of(w))
+
+
+def test_bounded_wait_reports_timeout_without_fault():
+    """A pipeline wait that can never complete gives up after its limit, sets
+    MOE_DEVERR_WAIT_TIMEOUT in the workspace's error word and returns; the
+    context stays usable (a layer call afterwards still matches the oracle)."""
+    ws = moe.alloc_workspace(4096)
+    moe.moe_selftest_bounded_wait(ws, 20_000_000)          # 20 ms
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == moe.DEVERR_WAIT_TIMEOUT
+    moe.moe_clear_device_error(ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    test_route_fed_scores_bit_exact(ROUTE_CASES[0])
