@@ -187,7 +187,7 @@ moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int
   const int bm = tc ? moe::tc_bm() : moe::simt_bm();
   const int bn_gu = tc ? moe::tc_cols_gateup() : moe::simt_bn();
   const int bn_dn = tc ? moe::tc_cols_down() : moe::simt_bn();
-  moe::launch_groups(offsets, a.E_r, a.E_s, a.T, bm, (a.f_r + bn_gu - 1) / bn_gu,
+  moe::launch_groups(offsets, a.E_r, a.E_s, a.T, bm, tc ? moe::tc_merge_rows() : 0, (a.f_r + bn_gu - 1) / bn_gu,
                      a.E_s ? (a.f_s + bn_gu - 1) / bn_gu : 0, (a.d + bn_dn - 1) / bn_dn,
                      (a.d + bn_dn - 1) / bn_dn, const_cast<int*>(a.grp_rows),
                      const_cast<int*>(a.grp_row0), const_cast<int*>(a.pre_gu),

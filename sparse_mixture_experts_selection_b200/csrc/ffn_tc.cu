@@ -21,6 +21,17 @@
 // MMA issuer (one thread), warps 2..5 = epilogue (TMEM -> registers -> global).
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the
 // epilogue of one unit overlaps the MMAs of the next.
+//
+// Short row tiles (an expert's last tile holding at most kSwapMaxRows rows) are
+// computed transposed: the weight tile is the M = 128 operand and the n rows
+// the N = round16(n) operand, D^T = W X^T, so the tensor cores do n/128 of a
+// full tile's work instead of padding the rows up to 128.  A tail of at most
+// kMergeMaxRows rows rides in the same unit as the full tile before it: each
+// stage then holds the full tile's rows, the tail's rows and ONE copy of the
+// weight tile, which feeds both the normal MMA and the transposed tail MMA.
+// Experts of a little more than 128 tokens -- the common case when T*K/E_r is
+// near 128 -- thus stream their weights through shared memory once, not twice,
+// and spend no MMAs on padding.  Such a unit holds both TMEM accumulators.
 #include <algorithm>
 #include <cuda.h>
 #include "common.cuh"
@@ -37,15 +48,22 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int kSwapMaxRows = 96;                // tiles of <= this many rows run transposed
+constexpr int kMergeMaxRows = 64;               // tails of <= this many rows join the tile before
+constexpr int A_SUB_ROWS = 32;                  // row box of the transposed tiles' token loads
+constexpr int A_SUB_BYTES = A_SUB_ROWS * BK * 2;
+constexpr int T_BYTES = kMergeMaxRows * BK * 2; // 8 KB: a merged tail's rows per stage
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * (STAGE_BYTES + T_BYTES) + 1024 + 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1, EPI_ROUTER = 2 };
 
 struct Params {
   CUtensorMap a_r, a_s;       // A: routed rows / shared rows
+  CUtensorMap a32_r, a32_s;   // the same with a 32-row box (transposed tiles)
   CUtensorMap b0_r, b1_r;     // routed B: gate & up (SWIGLU) or down (b0 only)
   CUtensorMap b0_s, b1_s;     // shared B
   const int* grp_rows;
@@ -71,11 +89,22 @@ struct Params {
 constexpr int UNIT_RING = 4;     // units handed from the producer to the MMA / epilogue warps
 
 // One work unit: group g (routed / shared), row tile, column tile and the
-// range of 64-wide k-blocks it reduces over.
+// range of 64-wide k-blocks it reduces over; n16 > 0 marks a transposed tile
+// (MMA N = n16); tail > 0 marks a full tile carrying the group's last tail
+// rows (transposed, MMA N = t16) in the same unit.
 struct Unit {
   int g, mt, nt, kb0, nk;
+  int rows, n16, tail, t16;
   bool sh;
 };
+
+// Row units of a group of `rows` rows: one per 128-row tile, except that a
+// last tile of at most kMergeMaxRows rows shares the unit of the tile before.
+__device__ __forceinline__ int row_units(int rows, int merge_max) {
+  const int mt = (rows + BM - 1) / BM;
+  const int last = rows - (mt - 1) * BM;
+  return mt - ((mt >= 2 && last <= merge_max) ? 1 : 0);
+}
 
 template <int EPI>
 __device__ __forceinline__ int total_units(const Params& p) {
@@ -96,6 +125,8 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
     w.kb0 = ks * p.r_per;
     w.nk = min(3 * p.r_nkd, w.kb0 + p.r_per) - w.kb0;
     w.nt = w.nt * p.r_ks + ks;          // packed (column tile, split) for the epilogue
+    w.rows = p.r_T;
+    w.n16 = w.tail = w.t16 = 0;
     return w;
   }
   int lo = 0, hi = p.G;                  // prefix[lo] <= u < prefix[lo + 1]
@@ -106,11 +137,17 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
   w.g = lo;
   w.sh = lo >= p.E_r;
   int local = u - __ldg(p.prefix + lo);
-  int mtiles = (__ldg(p.grp_rows + lo) + BM - 1) / BM;
-  w.mt = local % mtiles;
-  w.nt = local / mtiles;
+  w.rows = __ldg(p.grp_rows + lo);
+  const int runits = row_units(w.rows, kMergeMaxRows);
+  w.mt = local % runits;
+  w.nt = local / runits;
   w.kb0 = 0;
   w.nk = ((w.sh ? p.k_s : p.k_r) + BK - 1) / BK;
+  const int mtiles = (w.rows + BM - 1) / BM;
+  w.tail = (runits < mtiles && w.mt == runits - 1) ? w.rows - (mtiles - 1) * BM : 0;
+  w.t16 = (w.tail + 15) & ~15;
+  const int rv = min(BM, w.rows - w.mt * BM);
+  w.n16 = (w.tail == 0 && rv <= kSwapMaxRows) ? (rv + 15) & ~15 : 0;
   return w;
 }
 
@@ -125,6 +162,10 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int* 
 
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
+__device__ __forceinline__ uint16_t bf16_bits(float a) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(a));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -133,7 +174,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // Tensor-map coordinates of the A and B tiles of k-block i of unit w.
 template <int EPI>
 struct TileCoords {
-  const CUtensorMap *am, *b0, *b1;
+  const CUtensorMap *am, *am32, *b0, *b1;
   int ax, ay, bx, by;
 };
 
@@ -141,6 +182,7 @@ template <int EPI>
 __device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Unit& w, int i) {
   TileCoords<EPI> c;
   c.am = w.sh ? &p.a_s : &p.a_r;
+  c.am32 = w.sh ? &p.a32_s : &p.a32_r;
   c.b0 = w.sh ? &p.b0_s : &p.b0_r;
   c.b1 = w.sh ? &p.b1_s : &p.b1_r;
   int brow;
@@ -160,13 +202,44 @@ __device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Un
   return c;
 }
 
+// Epilogue of a transposed tile: the accumulator holds D^T, lane r = output
+// column colA (gate or first W_down half, columns [0, n16)) and colB (up or
+// second half, columns [128, 128 + n16)); accumulator column t = row row0 + t.
+// out0 points at output row row0.
+template <int EPI>
+__device__ __forceinline__ void epilogue_transposed(const Params& p, bool sh, uint16_t* out0, size_t row0,
+                                                    int rv, int n16, int colA, int ncols, uint32_t tb) {
+  const int colB = colA + BN / 2;                     // EPI_SCALE only
+#pragma unroll 1
+  for (int c = 0; c < n16; c += 32) {
+    float dv0[32], dv1[32];
+    tmem_ld32(tb + c, dv0);
+    tmem_ld32(tb + BN / 2 + c, dv1);
+#pragma unroll
+    for (int v = 0; v < 32; ++v) {
+      const int t = c + v;
+      if (t < rv) {
+        uint16_t* orow_p = out0 + (size_t)t * ncols;
+        if (EPI == EPI_SWIGLU) {
+          if (colA < ncols) orow_p[colA] = bf16_bits(silu(dv0[v]) * dv1[v]);
+        } else {
+          const float sc = (!sh && p.row_scale) ? __ldg(p.row_scale + row0 + t) : 1.0f;
+          if (colA < ncols) orow_p[colA] = bf16_bits(dv0[v] * sc);
+          if (colB < ncols) orow_p[colB] = bf16_bits(dv1[v] * sc);
+        }
+      }
+    }
+  }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sT = smem + STAGES * STAGE_BYTES;     // merged tails' rows
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (STAGE_BYTES + T_BYTES));
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -192,6 +265,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   if (warp == 1 && lane == 0) {
     prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.b0_r);
     prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
+    if (EPI != EPI_ROUTER) { prefetch_tmap(&p.a32_r); prefetch_tmap(&p.a32_s); }
   }
   tc_fence_before();
   __syncthreads();
@@ -217,11 +291,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
         if (u < 0) break;
         const Unit w = decode<EPI>(p, u);
+        // a transposed tile (and a merged tail) loads only the 32-row slices
+        // that hold its N rows
+        const int n_sub = w.n16 ? (w.n16 + A_SUB_ROWS - 1) / A_SUB_ROWS : 0;
+        const int t_sub = (w.t16 + A_SUB_ROWS - 1) / A_SUB_ROWS;
+        const uint32_t tx = (uint32_t)((n_sub ? n_sub * A_SUB_BYTES : A_BYTES) + t_sub * A_SUB_BYTES + B_BYTES);
         for (int i = 0; i < w.nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
           const TileCoords<EPI> c = tile_coords<EPI>(p, w, i);
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, c.am, &full[stage], c.ax, c.ay);
+          mbar_arrive_expect_tx(&full[stage], tx);
+          if (n_sub == 0) {
+            tma_load_2d(sA + stage * A_BYTES, c.am, &full[stage], c.ax, c.ay);
+          } else {
+            for (int q = 0; q < n_sub; ++q)
+              tma_load_2d(sA + stage * A_BYTES + q * A_SUB_BYTES, c.am32, &full[stage], c.ax,
+                          c.ay + q * A_SUB_ROWS);
+          }
+          for (int q = 0; q < t_sub; ++q)
+            tma_load_2d(sT + stage * T_BYTES + q * A_SUB_BYTES, c.am32, &full[stage], c.ax,
+                        c.ay + BM + q * A_SUB_ROWS);
           if (EPI == EPI_SWIGLU) {
             tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
             tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, c.b1, &full[stage], c.bx, c.by);
@@ -244,8 +332,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       // ---------------- MMA issuer ----------------
       int stage = 0;
       uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
+      int nb = 0;                           // accumulator buffer of the next one-buffer unit
+      uint32_t ph_e = 0;                    // bit b: phase of acc_empty[b]
       int slot = 0;
       uint32_t uphase = 0;
       for (;;) {
@@ -254,28 +342,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         mbar_arrive(&unit_empty[slot]);
         if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
         if (u < 0) break;
-        const int nk = decode<EPI>(p, u).nk;
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
+        const Unit w = decode<EPI>(p, u);
+        const int nk = w.nk;
+        // transposed tile: two M = 128 halves of the weight tile (gate | up, or
+        // the two 128-row halves of W_down's 256) against the N = n16 rows,
+        // into accumulator columns [0, n16) and [128, 128 + n16)
+        const uint32_t idesc_t = idesc_bf16_f32(BM, w.n16 ? w.n16 : 16);
+        const uint32_t idesc_tail = idesc_bf16_f32(BM, w.t16 ? w.t16 : 16);
+        // a unit with a merged tail holds buffer 0 (full tile) and buffer 1 (tail)
+        const bool two = w.tail > 0;
+        const int acc = two ? 0 : nb;
+        if (!mbar_wait(&acc_empty[acc], ((ph_e >> acc) & 1u) ^ 1u, abort_flag, p.err)) break;
+        ph_e ^= 1u << acc;
+        if (two) {
+          if (!mbar_wait(&acc_empty[1], ((ph_e >> 1) & 1u) ^ 1u, abort_flag, p.err)) break;
+          ph_e ^= 2u;
+        }
+        nb = two ? 0 : nb ^ 1;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tail = tmem_base + (uint32_t)BN;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {      // kb counts this unit's k-blocks
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+          if (w.n16 == 0) {
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2),
-                        sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), IDESC, (kb | k) != 0);
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2),
+                          sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), IDESC, (kb | k) != 0);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint64_t xd = sdesc_kmajor_sw128(a0 + k * UMMA_K * 2);
+              tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_t, (kb | k) != 0);
+              tc_mma_bf16(d_tmem + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
+                          idesc_t, (kb | k) != 0);
+            }
+          }
+          if (two) {
+            const uint32_t t0 = smem_u32(sT + stage * T_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint64_t xd = sdesc_kmajor_sw128(t0 + k * UMMA_K * 2);
+              tc_mma_bf16(d_tail, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_tail, (kb | k) != 0);
+              tc_mma_bf16(d_tail + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
+                          idesc_tail, (kb | k) != 0);
+            }
           }
           tc_commit(&empty[stage]);       // frees the stage once these MMAs are done
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit(&acc_full[acc]);        // accumulator ready for the epilogue
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (two) tc_commit(&acc_full[1]);
       }
       tc_commit(drain);                    // every MMA issued by this thread is done
       wait_drain(drain, 0, p.err);
@@ -284,8 +407,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     // ---------------- epilogue (warps 2..5) ----------------
     const int sub = warp & 3;              // TMEM lane quarter this warp may access
     const int r = sub * 32 + lane;         // row within the tile
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int nb = 0;                            // same buffer sequence as the MMA issuer
+    uint32_t ph_f = 0;                     // bit b: phase of acc_full[b]
     int slot = 0;
     uint32_t uphase = 0;
     for (;;) {
@@ -303,10 +426,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       const size_t orow = (EPI == EPI_ROUTER ? 0 : (size_t)__ldg(p.grp_row0 + w.g)) + m;
       const int ncols = sh ? p.ncols_s : p.ncols_r;
       uint16_t* out = (sh ? p.out_s : p.out_r) + orow * ncols;
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.err)) break;
+      const bool two = w.tail > 0;
+      const int acc = two ? 0 : nb;
+      nb = two ? 0 : nb ^ 1;
+      if (!mbar_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err)) break;
+      ph_f ^= 1u << acc;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == EPI_ROUTER) {
+      // transposed tiles: this thread owns output column(s) r of the unit and
+      // walks the rows along the accumulator columns
+      const int colA = EPI == EPI_SWIGLU ? nt * (BN / 2) + r : nt * BN + r;
+      const size_t row0 = orow - r;                       // output row of the tile's row 0
+      uint16_t* out0 = (sh ? p.out_s : p.out_r) + row0 * ncols;
+      if (EPI != EPI_ROUTER && w.n16) {
+        epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb);
+      } else if (EPI == EPI_ROUTER) {
         // fp32 partial logits of split (nt % ks) for experts of column tile nt / ks
         const int ks = nt % p.r_ks, ct = nt / p.r_ks;
         float* zrow = p.zpart + ((size_t)ks * p.r_T + m) * p.r_E;
@@ -368,8 +502,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (EPI != EPI_ROUTER && two) {
+        // the merged tail: rows (mt + 1) * 128 .. + tail, transposed, in buffer 1
+        if (!mbar_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err)) break;
+        ph_f ^= 2u;
+        tc_fence_after();
+        epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
+                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN);
+        tc_fence_before();
+        mbar_arrive(&acc_empty[1]);
+      }
     }
   }
 
@@ -416,6 +558,7 @@ static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
 }  // namespace tc
 
 int tc_bm() { return tc::BM; }
+int tc_merge_rows() { return tc::kMergeMaxRows; }
 int tc_cols_gateup() { return tc::BN / 2; }
 int tc_cols_down() { return tc::BN; }
 
@@ -522,6 +665,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
     const uint64_t wr_r = (uint64_t)a.E_r * a.f_r, wr_s = has_s ? (uint64_t)a.E_s * a.f_s : wr_r;
     ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM);
     ok &= make_tmap(&p.a_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d, BM);
+    ok &= make_tmap(&p.a32_r, a.x_r, (uint64_t)a.max_rows_r, a.d, A_SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d,
+                    A_SUB_ROWS);
     ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, BN / 2);
     ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, BN / 2);
     ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, BN / 2);
@@ -539,6 +685,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
     const uint64_t wd_rows_s = (uint64_t)(has_s ? a.E_s : a.E_r) * a.d;
     ok &= make_tmap(&p.a_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, BM);
     ok &= make_tmap(&p.a_s, has_s ? a.act_s : a.act_r, rows_s, fs, BM);
+    ok &= make_tmap(&p.a32_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, A_SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, has_s ? a.act_s : a.act_r, rows_s, fs, A_SUB_ROWS);
     ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
     ok &= make_tmap(&p.b1_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
     ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN);

@@ -31,7 +31,7 @@ void launch_hist(const int32_t* idx, int* hist, int chunk_shift, int T, int K, i
 void launch_counts(const int* hist, int n_chunks, int E, int* counts, cudaStream_t st);
 void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int* kept,
                  int* offsets, int* chunk_base, cudaStream_t st);
-void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
+void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int merge_max, int nt_gu_r, int nt_gu_s,
                    int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
                    int* pre_dn, int max_rows, int* err, int* tile_counters, cudaStream_t st);
 void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
@@ -66,6 +66,7 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
                              int E, int* err, int* ks_out, cudaStream_t st);
 
 int tc_bm();
+int tc_merge_rows();   // tails of <= this many rows share the unit of the tile before
 int tc_cols_gateup();
 int tc_cols_down();
 // which = 0: gate/up GEMM + SwiGLU epilogue; which = 1: down GEMM + gate scaling

@@ -336,7 +336,7 @@ scan_kernel(const int* __restrict__ hist, int n_chunks, int E, int cap, int* __r
 // (T rows each, row base j*T); unit prefixes for the two GEMMs, with tiles of
 // bm rows and nt_* column tiles per group.
 __global__ void __launch_bounds__(1024)
-groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, int nt_gu_r,
+groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, int merge_max, int nt_gu_r,
               int nt_gu_s, int nt_dn_r, int nt_dn_s, int* __restrict__ grp_rows,
               int* __restrict__ grp_row0, int* __restrict__ pre_gu, int* __restrict__ pre_dn,
               int max_rows, int* err, int* tile_counters) {
@@ -358,7 +358,10 @@ groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, 
     if (g < G) {
       if (g < E_r) { row0 = offsets[g]; rows = bad ? 0 : offsets[g + 1] - row0; }
       else { rows = bad ? 0 : T; row0 = (g - E_r) * T; }
+      // row units: one per bm-row tile; a last tile of <= merge_max rows
+      // shares the unit of the tile before it (tensor-core GEMM)
       int mt = (rows + bm - 1) / bm;
+      if (mt >= 2 && rows - (mt - 1) * bm <= merge_max) --mt;
       ugu = mt * (g < E_r ? nt_gu_r : nt_gu_s);
       udn = mt * (g < E_r ? nt_dn_r : nt_dn_s);
       grp_rows[g] = rows;
@@ -714,10 +717,10 @@ void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int
   scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, cap, counts, kept, offsets, chunk_base);
 }
 
-void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int nt_gu_r, int nt_gu_s,
+void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int merge_max, int nt_gu_r, int nt_gu_s,
                    int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
                    int* pre_dn, int max_rows, int* err, int* tile_counters, cudaStream_t st) {
-  groups_kernel<<<1, 1024, 0, st>>>(offsets, E_r, E_s, T, bm, nt_gu_r, nt_gu_s, nt_dn_r, nt_dn_s,
+  groups_kernel<<<1, 1024, 0, st>>>(offsets, E_r, E_s, T, bm, merge_max, nt_gu_r, nt_gu_s, nt_dn_r, nt_dn_s,
                                     grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err, tile_counters);
 }
 

@@ -33,6 +33,10 @@ SMALL = {
                                                         d_ffn=192, d_ffn_shared=136),
     "finegrained_small_cf": W["finegrained_64x1408_cf1.25"].with_(T=600, d_model=192, E_r=16, E_s=2,
                                                                   K=4, d_ffn=192, d_ffn_shared=136),
+    # ~110 rows per expert: full, partial (97..127 rows) and transposed short
+    # (<= 96 rows) tiles side by side
+    "finegrained_near_tile": W["finegrained_64x1408"].with_(T=440, d_model=192, E_r=16, E_s=2, K=4,
+                                                           d_ffn=192, d_ffn_shared=136),
     "deepseek_small": W["deepseek_v3"].with_(T=520, d_model=256, E_r=64, E_s=1, K=6, d_ffn=256,
                                              d_ffn_shared=384, n_groups=8, topk_groups=3),
     "decode_small": W["deepseek_v3_decode"].with_(T=24, d_model=320, E_r=64, d_ffn=128,
