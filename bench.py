@@ -18,6 +18,7 @@ sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -441,8 +442,12 @@ def run_ours(args, w, rank, world, local_rank):
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            rec = json.load(f).get("ffn_gate_up")
-        if rec:
+            doc = json.load(f)
+        rec = doc.get("ffn_gate_up")
+        src = os.path.join(ROOT, doc.get("source", ""))
+        # counters taken on another version of the kernel say nothing about this one
+        same = os.path.isfile(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == doc.get("source_sha256")
+        if rec and same:
             traffic = rec["ratio"] * gu_bytes
     layer = [layer_work(w, k) for k in kept_h]
     l_flops = float(np.mean([x[0] for x in layer]))
