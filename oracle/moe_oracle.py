@@ -52,6 +52,14 @@ reductions to a dense SwiGLU FFN computed with torch.nn.functional, a dense
 all-experts restatement of the layer equation, and planted-mistake tests.
 The expert FFN values themselves have no printed values on the pages: beyond
 those reductions they are "parity unpinned".
+
+Router losses and logging (aux_loss, z_loss, seq_balance_loss, load_entropy,
+dropped_rate) are pinned in tests/test_oracle_router_stats.py.  The e4m3
+quantization of expert weights and rows (e4m3_encode, pow2_scale,
+quantize_rows, swiglu_q8, layer_output_q8) is pinned in
+tests/test_oracle_fp8.py against torch's float8_e4m3fn conversion, ties to
+even, the closed form of the scale and the format's error bound; the
+quantized expert's values beyond that bound are "parity unpinned".
 """
 from __future__ import annotations
 
@@ -389,3 +397,107 @@ def load_entropy(counts: np.ndarray) -> float:
 def dropped_rate(kept: np.ndarray, counts: np.ndarray) -> float:
     """Fraction of (token, expert) pairs dropped by capacity, 1 - kept/selected."""
     return float(1.0 - np.sum(kept) / np.sum(counts))
+
+
+# ---------------------------------------------------------------------------
+# Expert weights in fewer bits ([GMF], "storing weights in fewer bits" for the
+# weight-streaming regime).  The pages name no format; the reading here (also
+# in the design notes): fp8 e4m3 codes (1 sign, 4 exponent bits with bias 7,
+# 3 mantissa bits, no infinities, largest finite 448) with one power-of-two
+# scale per weight row (output channel) and per activation row (token); the
+# tensor cores multiply e4m3 by e4m3, so the rows entering each GEMM are
+# quantized the same way.  A scale is the smallest power of two s with
+# amax / s <= 448, so x / s is exact and the only rounding is e4m3's own
+# (to nearest, ties to the even code, saturating at +-448).
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_table() -> np.ndarray:
+    """Values of the non-negative finite e4m3 codes 0..126 (ascending)."""
+    codes = np.arange(127)
+    e, m = codes >> 3, codes & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+
+
+def e4m3_encode(x32: np.ndarray) -> np.ndarray:
+    """uint8 e4m3 codes of fp32 values: nearest finite value, ties to the even
+    code, |x| >= 448 saturates to 448; the sign bit is x's (a negative value
+    that rounds to zero gives -0, code 0x80)."""
+    x = np.asarray(x32, np.float64)
+    tab = e4m3_table()
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(tab, a, side="left"), 0, 126)    # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - tab[lo], tab[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    sign = np.signbit(x).astype(np.uint8) << 7                      # -0 keeps its sign, as in IEEE
+    return (code | sign).astype(np.uint8)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, np.uint8)
+    v = e4m3_table()[np.minimum(c & 0x7F, 126)]
+    return np.where(c & 0x80, -v, v)
+
+
+def pow2_scale(amax32: np.ndarray) -> np.ndarray:
+    """Smallest power of two s with amax / s <= 448, as fp32 (1 where amax == 0).
+    With amax = M * 2^E (1 <= M < 2): s = 2^(E - 8 + [M > 1.75])."""
+    a = np.asarray(amax32, np.float64)
+    m, ex = np.frexp(a)                     # a = m * 2^ex, 0.5 <= m < 1
+    e = (ex - 1) - 8 + (2.0 * m > 1.75)
+    return np.where(a > 0, np.ldexp(1.0, e), 1.0).astype(F32)
+
+
+def quantize_rows(x32: np.ndarray):
+    """Per-row power-of-two scale and e4m3 codes of an fp32 matrix [n, c]."""
+    x = np.asarray(x32, F32)
+    s = pow2_scale(np.max(np.abs(x), axis=1) if x.shape[1] else np.zeros(x.shape[0], F32))
+    codes = e4m3_encode(x.astype(np.float64) / s.astype(np.float64)[:, None])
+    return codes, s
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    return e4m3_decode(codes) * np.asarray(scales, np.float64)[:, None]
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round to bf16 (to nearest even) through torch's conversion; float64 out."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(x, np.float64)))
+    return t.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def swiglu_q8(x: np.ndarray, wg, wu, wd) -> np.ndarray:
+    """One SwiGLU expert with e4m3 weights: wg, wu, wd are (codes, scales) with
+    the nn.Linear layout.  The input rows are quantized per row, the products
+    accumulate in float64, the SwiGLU product A is stored in bf16 and quantized
+    per row before the down projection."""
+    xq = dequantize_rows(*quantize_rows(np.asarray(x, F32)))
+    u = xq @ dequantize_rows(*wg).T
+    v = xq @ dequantize_rows(*wu).T
+    with np.errstate(over="ignore"):
+        a = bf16_round(u / (1.0 + np.exp(-u)) * v)
+    aq = dequantize_rows(*quantize_rows(a.astype(F32)))
+    return aq @ dequantize_rows(*wd).T
+
+
+def layer_output_q8(cfg: LayerConfig, h: np.ndarray, idx: np.ndarray, gates: np.ndarray,
+                    disp: Dispatch, weights, tokens: Optional[np.ndarray] = None) -> np.ndarray:
+    """layer_output with e4m3 expert weights; ``weights(which, ex)`` returns
+    (codes, scales).  Same layer equation, experts evaluated by swiglu_q8."""
+    tok = np.arange(cfg.T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    x = np.asarray(h, np.float64)[tok]
+    y = x * float(cfg.add_residual)
+    for j in range(cfg.E_s):
+        y = y + swiglu_q8(x, weights("sgate", j), weights("sup", j), weights("sdown", j))
+    kept = disp.row_of[tok] >= 0
+    ex_of = idx[tok].astype(np.int64)
+    for ex in np.unique(ex_of[kept]):
+        rows, ks = np.nonzero((ex_of == ex) & kept)
+        o = swiglu_q8(x[rows], weights("gate", ex), weights("up", ex), weights("down", ex))
+        y[rows] += gates[tok[rows], ks].astype(np.float64)[:, None] * o
+    return y
