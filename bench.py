@@ -61,9 +61,13 @@ def layer_work(w, kept: np.ndarray):
     touched = int((kept > 0).sum())
     d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
     flops = 2 * d * w.E_r * w.T + 6 * d * f * n_rows + 6 * d * fs * w.E_s * w.T
-    es = 2 if w.dtype == "bf16" else 4
-    nbytes = (touched * 3 * d * f * es + w.E_s * 3 * d * fs * es + w.E_r * d * 4
-              + 2 * w.T * d * es)
+    es = 2 if w.dtype != "f32" else 4
+    if w.dtype == "bf16_e4m3":
+        # one byte per weight plus one fp32 scale per weight row
+        wbytes = touched * (3 * d * f + 4 * (2 * f + d)) + w.E_s * (3 * d * fs + 4 * (2 * fs + d))
+    else:
+        wbytes = touched * 3 * d * f * es + w.E_s * 3 * d * fs * es
+    nbytes = wbytes + w.E_r * d * 4 + 2 * w.T * d * es
     return flops, nbytes
 
 
@@ -76,8 +80,14 @@ def gateup_work(w, kept: np.ndarray):
     d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
     rows_s = w.E_s * w.T
     flops = 4 * d * (f * n_rows + fs * rows_s)
-    nbytes = 2 * (touched * 2 * d * f + w.E_s * 2 * d * fs + (n_rows + min(rows_s, w.T)) * d
-                  + n_rows * f + rows_s * fs)
+    if w.dtype == "bf16_e4m3":
+        # e4m3 weights and rows (+ fp32 row scales), bf16 SwiGLU products out
+        x_rows = n_rows + min(rows_s, w.T)
+        nbytes = (touched * 2 * (d * f + 4 * f) + w.E_s * 2 * (d * fs + 4 * fs) + x_rows * (d + 4)
+                  + 2 * (n_rows * f + rows_s * fs))
+    else:
+        nbytes = 2 * (touched * 2 * d * f + w.E_s * 2 * d * fs + (n_rows + min(rows_s, w.T)) * d
+                      + n_rows * f + rows_s * fs)
     return flops, nbytes
 
 
@@ -87,7 +97,11 @@ def down_work(w, kept: np.ndarray):
     d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
     rows_s = w.E_s * w.T
     flops = 2 * d * (f * n_rows + fs * rows_s)
-    nbytes = 2 * (touched * d * f + w.E_s * d * fs + n_rows * f + rows_s * fs + (n_rows + rows_s) * d)
+    if w.dtype == "bf16_e4m3":
+        nbytes = (touched * (d * f + 4 * d) + w.E_s * (d * fs + 4 * d) + n_rows * (f + 4)
+                  + rows_s * (fs + 4) + 2 * (n_rows + rows_s) * d)
+    else:
+        nbytes = 2 * (touched * d * f + w.E_s * d * fs + n_rows * f + rows_s * fs + (n_rows + rows_s) * d)
     return flops, nbytes
 
 
@@ -292,7 +306,8 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    bf16 = w.dtype == "bf16"
+    bf16 = w.dtype != "f32"                 # bf16 activations (bf16 and e4m3-weight layers)
+    e4m3 = w.dtype == "bf16_e4m3"
     dt = torch.bfloat16 if bf16 else torch.float32
 
     # ---- inputs resident in HBM ----
@@ -304,6 +319,13 @@ def run_ours(args, w, rank, world, local_rank):
             continue
         t = torch.empty((n, rows, cols), dtype=dt, device=dev)
         native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, tid, 0, sigma, stream=stream.cuda_stream)
+        if e4m3:
+            # the same bf16 weights as e4m3 blobs (codes + row scales); the bf16 copy is dropped
+            q = torch.empty(moe.moe_quantized_bytes(n * rows, cols), dtype=torch.uint8, device=dev)
+            moe.moe_quantize_rows(t, moe.DTYPE_BF16, n * rows, cols, q, stream=stream)
+            stream.synchronize()
+            del t
+            t = q
         W[k] = t
     e = torch.from_numpy(mi.gen_centroids(w)).to(dev)
     b = torch.from_numpy(mi.gen_bias(w)).to(dev)
@@ -447,26 +469,29 @@ def run_ours(args, w, rank, world, local_rank):
         src = os.path.join(ROOT, doc.get("source", ""))
         # counters taken on another version of the kernel say nothing about this one
         same = os.path.isfile(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == doc.get("source_sha256")
-        if rec and same:
+        if rec and same and w.dtype == "bf16":       # counters of the bf16 kernel
             traffic = rec["ratio"] * gu_bytes
     layer = [layer_work(w, k) for k in kept_h]
     l_flops = float(np.mean([x[0] for x in layer]))
     l_bytes = float(np.mean([x[1] for x in layer]))
-    t_roof = max(l_flops / (bf16_peak * 1e12), l_bytes / (hbm * 1e9))
+    # e4m3 tensor-core peak: the measured bf16 figure x the nominal fp8/bf16 ratio (4.5 / 2.25)
+    mma_peak = bf16_peak * (2.0 if e4m3 else 1.0)
+    t_roof = max(l_flops / (mma_peak * 1e12), l_bytes / (hbm * 1e9))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if bf16 else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if e4m3 else ("bf16" if bf16 else "f32"),
         "data": "synthetic", "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "kernel": "ffn_gate_up (tcgen05 grouped GEMM)",
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "tensor_tflops": gu_flops / gu_s / 1e12,
-                     "tensor_frac_sustained": gu_flops / gu_s / 1e12 / bf16_peak},
+                     "tensor_frac_sustained": gu_flops / gu_s / 1e12 / mma_peak},
         "layer_roofline": {"t_roof_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms_per_step,
                            "flops": l_flops, "bytes": l_bytes,
-                           "bound": "hbm" if l_bytes / (hbm * 1e9) >= l_flops / (bf16_peak * 1e12) else "tensor",
-                           "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained"},
+                           "bound": "hbm" if l_bytes / (hbm * 1e9) >= l_flops / (mma_peak * 1e12) else "tensor",
+                           "peaks": f"{peak_kind}: {hbm} GB/s, {mma_peak} TFLOP/s sustained"
+                                    + (" (e4m3: bf16 x 2, nominal ratio)" if e4m3 else "")},
         "phases_ms": {p: float(np.mean(phase_ms[:, i])) for i, p in enumerate(moe.PHASES)},
         "down_gemm": {"achieved_gbs": float(np.mean([x[1] for x in dn])) / (float(np.mean(dn_ms)) / 1000) / 1e9},
         "rows_per_step": float(np.mean(kept_h.sum(1))),
@@ -476,7 +501,10 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clocks.summary(),
         # our kernels per step: [centroid split + router GEMM | CUDA-core logits], select,
         # scan, scatter, gather, group tables, gate/up GEMM, down GEMM, combine, bias step
-        "gpu_launches": (11 if bf16 else 10) * args.steps,
+        # per step: split, router GEMM, select, scan, scatter, gather (e4m3: gather +
+        # quantize), groups, gate/up, down, combine, bias; e4m3 adds the quantization
+        # of A, and of h and the shared A when there are shared experts
+        "gpu_launches": ((11 if bf16 else 10) + ((1 + 2 * (w.E_s > 0)) if e4m3 else 0)) * args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)

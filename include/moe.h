@@ -32,6 +32,13 @@
  *    aligned; the workspace 256-byte aligned.
  *  - Activations and expert weights have the element type cfg->dtype
  *    (MOE_DTYPE_F32: float; MOE_DTYPE_BF16: bfloat16 bits in uint16).
+ *    MOE_DTYPE_BF16_E4M3: activations bf16, expert weights e4m3 blobs: an
+ *    [n, rows, cols] weight tensor is n*rows*cols bytes of e4m3 codes (1 sign,
+ *    4 exponent bits with bias 7, 3 mantissa bits, largest finite 448) followed
+ *    by n*rows float32 row scales (powers of two); weight (i, r, c) is
+ *    code[(i*rows + r)*cols + c] * scale[i*rows + r].  moe_quantize_rows writes
+ *    this layout from bf16 or fp32 weights; d_model, d_ffn and d_ffn_shared
+ *    must be multiples of 16.
  *    Centroids e, biases b, scores and gates are always float32; indices and
  *    counts are int32.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
@@ -72,7 +79,14 @@ typedef enum {
 } moe_status;
 
 enum { MOE_SCORE_SIGMOID = 0, MOE_SCORE_SOFTMAX = 1 };
-enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+enum {
+  MOE_DTYPE_F32 = 0,
+  MOE_DTYPE_BF16 = 1,
+  /* bf16 activations (h, y, x, slots, shared_out) with e4m3 expert weights: each
+   * weight pointer is an e4m3 blob (moe_quantize_rows), and the rows entering
+   * the two expert GEMMs are quantized the same way inside the library */
+  MOE_DTYPE_BF16_E4M3 = 2
+};
 
 /* device error word values (moe_get_device_error) */
 enum {
@@ -94,7 +108,7 @@ typedef struct {
   int32_t topk_groups;   /* groups kept per token                                       */
   int32_t group_topn;    /* a group's score = sum of its top group_topn keys (0 = none) */
   float capacity_factor; /* <= 0: dropless; else C = floor(T*K*CF/E_r) rows per expert  */
-  int32_t dtype;         /* MOE_DTYPE_F32 or MOE_DTYPE_BF16                             */
+  int32_t dtype;         /* MOE_DTYPE_F32, MOE_DTYPE_BF16 or MOE_DTYPE_BF16_E4M3         */
   int32_t add_residual;  /* 1: y includes h_t                                           */
 } moe_config;
 
@@ -247,6 +261,26 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
  *   ws: at least moe_router_stats_workspace_size bytes (its first 256 bytes
  *   are not used by this call).  Deterministic (no floating-point atomics).
  */
+/*
+ * Expert weights in fewer bits ("GPUs, memory and failures", serving notes:
+ * storing weights in fewer bits for the weight-streaming regime; the pages
+ * fix no format -- this is the library's): e4m3 codes with one power-of-two
+ * scale per row, the smallest s with max_c |x[r][c]| / s <= 448 (at least
+ * 2^-126; 1 for an all-zero row), each element x / s rounded to the nearest
+ * e4m3 value, ties to the even code, saturating at +-448.
+ *
+ * moe_quantized_bytes: size of the blob for n_rows x cols (cols a positive
+ *   multiple of 16): n_rows*cols code bytes + n_rows*4 scale bytes.
+ * moe_quantize_rows: src [n_rows, cols] (src_dtype MOE_DTYPE_BF16 or
+ *   MOE_DTYPE_F32, 16-byte aligned, finite values) -> dst blob (16-byte
+ *   aligned, moe_quantized_bytes long).  Deterministic, bit-exact with the
+ *   definition above.  For the e4m3 layers quantize each weight tensor as
+ *   n_rows = experts * rows.
+ */
+moe_status moe_quantized_bytes(int64_t n_rows, int32_t cols, size_t* bytes);
+moe_status moe_quantize_rows(const void* src, int32_t src_dtype, int64_t n_rows, int32_t cols, void* dst,
+                             void* stream);
+
 moe_status moe_router_stats_workspace_size(const moe_config* cfg, int32_t seq_len, size_t* bytes);
 moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* z, const int32_t* idx,
                             const int32_t* kept, int32_t seq_len, float alpha_aux, float c_z,

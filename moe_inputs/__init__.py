@@ -138,7 +138,7 @@ class Workload:
     d_ffn: int
     d_ffn_shared: int
     score_fn: int          # 0 = sigmoid affinity, 1 = softmax
-    dtype: str             # "f32" or "bf16"
+    dtype: str             # "f32", "bf16", or "bf16_e4m3" (bf16 activations, e4m3 expert weights)
     seed: int
     n_groups: int = 1
     topk_groups: int = 1
@@ -184,10 +184,15 @@ WORKLOADS = {
 # The fine-grained layer is also run with GShard capacity factor 1.25.
 WORKLOADS["finegrained_64x1408_cf1.25"] = WORKLOADS["finegrained_64x1408"].with_(
     name="finegrained_64x1408_cf1.25", capacity_factor=1.25)
+# The DeepSeek-V3 layers with e4m3 expert weights (the same bf16 weights,
+# quantized per row): the weight-streaming regime with half the bytes.
+WORKLOADS["deepseek_v3_e4m3"] = WORKLOADS["deepseek_v3"].with_(name="deepseek_v3_e4m3", dtype="bf16_e4m3")
+WORKLOADS["deepseek_v3_decode_e4m3"] = WORKLOADS["deepseek_v3_decode"].with_(
+    name="deepseek_v3_decode_e4m3", dtype="bf16_e4m3")
 
 
 def _dtype_round(x: np.ndarray, dtype: str) -> np.ndarray:
-    return round_bf16(x) if dtype == "bf16" else x
+    return round_bf16(x) if dtype != "f32" else x
 
 
 def gen_h(w: Workload, step: int = 0, tokens: Optional[slice] = None) -> np.ndarray:

@@ -72,5 +72,5 @@ def weight_host(w: Workload, which: str, expert: int, threads: int = 0) -> np.nd
     from . import bf16_bits_to_f32
     tid, n, rows, cols, sigma = weight_spec(w, which)
     per = rows * cols
-    x = fill_host(per, w.dtype == "bf16", w.seed, tid, expert * per, sigma, threads=threads)
-    return (bf16_bits_to_f32(x) if w.dtype == "bf16" else x).reshape(rows, cols)
+    x = fill_host(per, w.dtype != "f32", w.seed, tid, expert * per, sigma, threads=threads)
+    return (bf16_bits_to_f32(x) if w.dtype != "f32" else x).reshape(rows, cols)

@@ -444,11 +444,12 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
 
 
 def pow2_scale(amax32: np.ndarray) -> np.ndarray:
-    """Smallest power of two s with amax / s <= 448, as fp32 (1 where amax == 0).
-    With amax = M * 2^E (1 <= M < 2): s = 2^(E - 8 + [M > 1.75])."""
+    """Smallest power of two s with amax / s <= 448, as fp32 (1 where amax == 0),
+    and never below 2^-126 (a scale is a normal fp32 number).
+    With amax = M * 2^E (1 <= M < 2): s = 2^max(E - 8 + [M > 1.75], -126)."""
     a = np.asarray(amax32, np.float64)
     m, ex = np.frexp(a)                     # a = m * 2^ex, 0.5 <= m < 1
-    e = (ex - 1) - 8 + (2.0 * m > 1.75)
+    e = np.maximum((ex - 1) - 8 + (2.0 * m > 1.75), -126)
     return np.where(a > 0, np.ldexp(1.0, e), 1.0).astype(F32)
 
 

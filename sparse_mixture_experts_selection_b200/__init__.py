@@ -22,12 +22,13 @@ __all__ = [
     "moe_expert_ffn", "moe_expert_ffn_workspace_size", "moe_combine", "moe_bias_update",
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
     "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
+    "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3",
     "moe_set_phase_events", "moe_selftest_bounded_wait",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
 
 SCORE_SIGMOID, SCORE_SOFTMAX = 0, 1
-DTYPE_F32, DTYPE_BF16 = 0, 1
+DTYPE_F32, DTYPE_BF16, DTYPE_BF16_E4M3 = 0, 1, 2
 DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_INDEX = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
@@ -69,6 +70,8 @@ SIGNATURES = {
                                          _P, _P, _P, _P, _I32, ctypes.c_float, _P, _P,
                                          ctypes.c_size_t, _P]),
     "moe_router_stats_workspace_size": (ctypes.c_int, [_P, _I32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_quantized_bytes": (ctypes.c_int, [ctypes.c_int64, _I32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_quantize_rows": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _I32, _P, _P]),
     "moe_router_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "moe_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
@@ -123,7 +126,8 @@ def config_for(w, **overrides) -> MoeConfig:
     c = MoeConfig(T=w.T, d_model=w.d_model, E_r=w.E_r, E_s=w.E_s, K=w.K, d_ffn=w.d_ffn,
                   d_ffn_shared=w.d_ffn_shared, score_fn=w.score_fn, n_groups=w.n_groups,
                   topk_groups=w.topk_groups, group_topn=w.group_topn,
-                  capacity_factor=w.capacity_factor, dtype=DTYPE_BF16 if w.dtype == "bf16" else DTYPE_F32,
+                  capacity_factor=w.capacity_factor,
+                  dtype={"bf16": DTYPE_BF16, "bf16_e4m3": DTYPE_BF16_E4M3}.get(w.dtype, DTYPE_F32),
                   add_residual=w.add_residual)
     for k, v in overrides.items():
         setattr(c, k, v)
@@ -161,6 +165,17 @@ def moe_router_stats_workspace_size(cfg: MoeConfig, seq_len: int = 0) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().moe_router_stats_workspace_size(ctypes.byref(cfg), int(seq_len), ctypes.byref(n)))
     return n.value
+
+
+def moe_quantized_bytes(n_rows: int, cols: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_quantized_bytes(int(n_rows), int(cols), ctypes.byref(n)))
+    return n.value
+
+
+def moe_quantize_rows(src, src_dtype: int, n_rows: int, cols: int, dst, stream=None):
+    _check(lib().moe_quantize_rows(_ptr(src), int(src_dtype), int(n_rows), int(cols), _ptr(dst),
+                                   _stream(stream)))
 
 
 # order of the values moe_router_stats writes

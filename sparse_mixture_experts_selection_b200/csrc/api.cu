@@ -25,7 +25,11 @@ constexpr int kChunkShift = 8;          // histogram chunk = 256 tokens (the sca
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
-size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+// bytes of an activation element (h, y, x_perm, A, slots): bf16 for the bf16
+// and e4m3-weight layers, fp32 for fp32 layers
+size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_F32 ? 4 : 2; }
+int act_dtype(int dtype) { return dtype == MOE_DTYPE_F32 ? MOE_DTYPE_F32 : MOE_DTYPE_BF16; }
+bool is_q8(int dtype) { return dtype == MOE_DTYPE_BF16_E4M3; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t capacity_rows(const moe_config& c) {
@@ -39,6 +43,9 @@ int64_t capacity_rows(const moe_config& c) {
 struct Layout {
   size_t err, scores, hist, chunk_base, counts, kept, offsets, grp_rows, grp_row0, pre_gu, pre_dn;
   size_t idx, gates, row_of, perm_tok, row_gate, maxvio, x_perm, act_r, act_s, slot_r, slot_s, e3;
+  // e4m3-weight layers: row scales of x_perm (codes), the e4m3 copy of h and its
+  // scales (shared experts), the e4m3 copies of A and their scales
+  size_t xs, hq, hs, actq_r, actq_s, as_r, as_s;
   size_t total;
   int n_chunks;
   int64_t cap, R;
@@ -57,8 +64,9 @@ Layout make_layout(const moe_config& c) {
   L.err = take(kAlign);
   // fp32 logits: split-K partial sums of the tensor-core router (bf16 layers)
   // or the CUDA-core logits (fp32 layers)
-  L.scores = take((size_t)(c.dtype == MOE_DTYPE_BF16 ? moe::kRouterMaxSplits : 1) * c.T * c.E_r * 4);
-  L.e3 = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)3 * c.E_r * c.d_model * 2 : 0);
+  const bool tcr = c.dtype != MOE_DTYPE_F32;          // tensor-core router
+  L.scores = take((size_t)(tcr ? moe::kRouterMaxSplits : 1) * c.T * c.E_r * 4);
+  L.e3 = take(tcr ? (size_t)3 * c.E_r * c.d_model * 2 : 0);
   L.hist = take((size_t)L.n_chunks * c.E_r * 4);
   L.chunk_base = take((size_t)L.n_chunks * c.E_r * 4);
   L.counts = take((size_t)c.E_r * 4);
@@ -74,11 +82,20 @@ Layout make_layout(const moe_config& c) {
   L.perm_tok = take((size_t)L.R * 4);
   L.row_gate = take((size_t)L.R * 4);
   L.maxvio = take(4);
-  L.x_perm = take((size_t)L.R * c.d_model * es);
+  const bool q8 = is_q8(c.dtype);
+  const size_t fs = c.E_s ? c.d_ffn_shared : 0;
+  L.x_perm = take((size_t)L.R * c.d_model * (q8 ? 1 : es));
   L.act_r = take((size_t)L.R * c.d_ffn * es);
-  L.act_s = take((size_t)c.E_s * c.T * (c.E_s ? c.d_ffn_shared : 0) * es);
+  L.act_s = take((size_t)c.E_s * c.T * fs * es);
   L.slot_r = take((size_t)L.R * c.d_model * es);
   L.slot_s = take((size_t)c.E_s * c.T * c.d_model * es);
+  L.xs = take(q8 ? (size_t)L.R * 4 : 0);
+  L.hq = take(q8 && c.E_s ? (size_t)c.T * c.d_model : 0);
+  L.hs = take(q8 && c.E_s ? (size_t)c.T * 4 : 0);
+  L.actq_r = take(q8 ? (size_t)L.R * c.d_ffn : 0);
+  L.actq_s = take(q8 ? (size_t)c.E_s * c.T * fs : 0);
+  L.as_r = take(q8 ? (size_t)L.R * 4 : 0);
+  L.as_s = take(q8 ? (size_t)c.E_s * c.T * 4 : 0);
   L.total = o;
   return L;
 }
@@ -99,7 +116,8 @@ moe_status validate(const moe_config* cfg) {
     return fail(MOE_ERR_INVALID_ARG, "d_ffn_shared=%d must be a positive multiple of 8", c.d_ffn_shared);
   if (c.score_fn != MOE_SCORE_SIGMOID && c.score_fn != MOE_SCORE_SOFTMAX)
     return fail(MOE_ERR_INVALID_ARG, "score_fn=%d", c.score_fn);
-  if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c.dtype);
+  if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16 && c.dtype != MOE_DTYPE_BF16_E4M3)
+    return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c.dtype);
   if (c.add_residual != 0 && c.add_residual != 1) return fail(MOE_ERR_INVALID_ARG, "add_residual=%d", c.add_residual);
   if (!std::isfinite(c.capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is not finite");
   if (c.n_groups < 1) return fail(MOE_ERR_INVALID_ARG, "n_groups=%d < 1", c.n_groups);
@@ -114,8 +132,10 @@ moe_status validate(const moe_config* cfg) {
     if (c.group_topn > gsz) return fail(MOE_ERR_INVALID_ARG, "group_topn=%d > group size %d", c.group_topn, gsz);
     if (c.n_groups > 32) return fail(MOE_ERR_UNSUPPORTED, "n_groups=%d > 32", c.n_groups);
   }
-  if (c.dtype == MOE_DTYPE_BF16 && (c.d_model < 64 || c.d_ffn < 64 || (c.E_s > 0 && c.d_ffn_shared < 64)))
+  if (c.dtype != MOE_DTYPE_F32 && (c.d_model < 64 || c.d_ffn < 64 || (c.E_s > 0 && c.d_ffn_shared < 64)))
     return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d_model, d_ffn, d_ffn_shared >= 64");
+  if (is_q8(c.dtype) && (c.d_model % 16 || c.d_ffn % 16 || (c.E_s > 0 && c.d_ffn_shared % 16)))
+    return fail(MOE_ERR_UNSUPPORTED, "e4m3 weights need d_model, d_ffn, d_ffn_shared multiples of 16");
   return MOE_OK;
 }
 
@@ -143,7 +163,7 @@ template <typename T> T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-bool use_tensor_cores(int dtype) { return dtype == MOE_DTYPE_BF16; }
+bool use_tensor_cores(int dtype) { return dtype != MOE_DTYPE_F32; }
 
 // a1-a4: logits (tensor cores for bf16, CUDA cores for fp32) unless scores are
 // fed, then activation, selection, gates and the per-chunk histogram.
@@ -200,6 +220,14 @@ moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int
     } else {
       moe::launch_ffn_simt(a, which, st);
     }
+    if (which == 0 && a.q8) {
+      // the down GEMM multiplies e4m3 by e4m3: quantize the SwiGLU output rows
+      moe::launch_quantize_rows(a.act_r, MOE_DTYPE_BF16, nullptr, 0, offsets + a.E_r, max_rows, a.f_r,
+                                static_cast<uint8_t*>(a.actq_r), a.as_r, a.err, st);
+      if (a.E_s)
+        moe::launch_quantize_rows(a.act_s, MOE_DTYPE_BF16, nullptr, 0, nullptr, (int64_t)a.E_s * a.T, a.f_s,
+                                  static_cast<uint8_t*>(a.actq_s), a.as_s, a.err, st);
+    }
     if (phase_base >= 0 && which == 0) mark_phase(phase_base + 1, st);
   }
   return cuda_status();
@@ -239,11 +267,19 @@ moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_expert
   if (n_experts < 1 || n_experts > 1024) return fail(MOE_ERR_INVALID_ARG, "n_experts=%d outside [1, 1024]", n_experts);
   if (d_ffn < 8 || d_ffn % 8) return fail(MOE_ERR_INVALID_ARG, "d_ffn=%d must be a positive multiple of 8", d_ffn);
   if (max_rows < 0) return fail(MOE_ERR_INVALID_ARG, "max_rows=%d < 0", max_rows);
+  if (is_q8(cfg->dtype) && d_ffn % 16) return fail(MOE_ERR_UNSUPPORTED, "e4m3 weights need d_ffn % 16 == 0");
+  const size_t mr = (size_t)(max_rows < 1 ? 1 : max_rows);
   size_t o = 0;
   o = align_up(o + kAlign);                                  // error word
   o = align_up(o + (size_t)n_experts * 8);                    // grp_rows, grp_row0
   o = align_up(o + (size_t)(n_experts + 1) * 8);              // pre_gu, pre_dn
-  o = align_up(o + (size_t)(max_rows < 1 ? 1 : max_rows) * d_ffn * elem_bytes(cfg->dtype));
+  o = align_up(o + mr * d_ffn * elem_bytes(cfg->dtype));     // A
+  if (is_q8(cfg->dtype)) {
+    o = align_up(o + mr * cfg->d_model);                      // e4m3 x
+    o = align_up(o + mr * 4);                                 // its row scales
+    o = align_up(o + mr * d_ffn);                             // e4m3 A
+    o = align_up(o + mr * 4);                                 // its row scales
+  }
   *bytes = o;
   return MOE_OK;
 }
@@ -299,7 +335,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ff
   size_t need = 0;
   MOE_CHECK(moe_expert_ffn_workspace_size(cfg, n_experts, d_ffn, max_rows, &need));
   const moe_config& c = *cfg;
-  if (c.dtype == MOE_DTYPE_BF16 && d_ffn < 64) return fail(MOE_ERR_UNSUPPORTED, "bf16 needs d_ffn >= 64");
+  if (c.dtype != MOE_DTYPE_F32 && d_ffn < 64) return fail(MOE_ERR_UNSUPPORTED, "bf16 needs d_ffn >= 64");
   MOE_NONNULL4(offsets); MOE_NONNULL(x); MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down);
   MOE_NONNULL(out); MOE_ALIGNED4(row_scale);
   MOE_CHECK(check_ws(ws, ws_bytes, need));
@@ -324,6 +360,20 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_experts, int32_t d_ff
   a.out_r = out; a.out_s = out;
   a.err = at<int>(ws, 0);
   a.tile_counters = at<int>(ws, 64);   // spare words of the error block
+  if (is_q8(c.dtype)) {
+    const size_t mr = (size_t)max_rows;
+    o = align_up(o + mr * d_ffn * elem_bytes(c.dtype));
+    uint8_t* xq = at<uint8_t>(ws, o); o = align_up(o + mr * c.d_model);
+    float* xs = at<float>(ws, o);     o = align_up(o + mr * 4);
+    a.actq_r = a.actq_s = at<void>(ws, o); o = align_up(o + mr * d_ffn);
+    a.as_r = a.as_s = at<float>(ws, o);
+    // rows 0 .. offsets[n_experts] of x, quantized for the e4m3 gate/up GEMM
+    moe::launch_quantize_rows(x, MOE_DTYPE_BF16, nullptr, 0, offsets + n_experts, max_rows, c.d_model,
+                              xq, xs, a.err, st);
+    a.q8 = 1;
+    a.x_r = a.x_s = xq;
+    a.xs_r = a.xs_s = xs;
+  }
   return run_ffn(c, a, offsets, max_rows, st);
 }
 
@@ -334,7 +384,7 @@ moe_status moe_combine(const moe_config* cfg, const void* h, const void* slot,
   MOE_NONNULL(h); MOE_NONNULL(slot); MOE_NONNULL4(row_of); MOE_NONNULL(y);
   if (c.E_s > 0) MOE_NONNULL(shared_out);
   moe::launch_combine(h, slot, shared_out, row_of, y, c.T, c.d_model, c.K, c.E_s, c.add_residual,
-                      c.dtype, 0x7FFFFFFF, static_cast<cudaStream_t>(stream));
+                      act_dtype(c.dtype), 0x7FFFFFFF, static_cast<cudaStream_t>(stream));
   return cuda_status();
 }
 
@@ -392,7 +442,18 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   moe::launch_scatter(idx, gates, offsets, at<int>(ws, L.chunk_base), (int)L.cap, c.T, c.K, c.E_r,
                       perm_tok, row_of, row_gate, err, st);
   void* x_perm = at<void>(ws, L.x_perm);
-  moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model, (int)es, (int)L.R, c.T, err, st);
+  const bool q8 = is_q8(c.dtype);
+  if (q8) {
+    // gather + quantize: e4m3 rows of x_perm with their scales, and of h for
+    // the shared experts
+    moe::launch_quantize_rows(h, MOE_DTYPE_BF16, perm_tok, c.T, offsets + c.E_r, L.R, c.d_model,
+                              static_cast<uint8_t*>(x_perm), at<float>(ws, L.xs), err, st);
+    if (c.E_s)
+      moe::launch_quantize_rows(h, MOE_DTYPE_BF16, nullptr, 0, nullptr, c.T, c.d_model,
+                                at<uint8_t>(ws, L.hq), at<float>(ws, L.hs), err, st);
+  } else {
+    moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model, (int)es, (int)L.R, c.T, err, st);
+  }
   mark_phase(2, st);
   // a6-a7: grouped SwiGLU experts (routed + shared) with gate-scaled outputs
   moe::FfnArgs a{};
@@ -409,11 +470,19 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   a.out_r = at<void>(ws, L.slot_r); a.out_s = c.E_s ? at<void>(ws, L.slot_s) : a.out_r;
   a.err = err;
   a.tile_counters = err + 16;          // spare words of the error block
+  if (q8) {
+    a.q8 = 1;
+    a.x_s = c.E_s ? at<void>(ws, L.hq) : x_perm;
+    a.xs_r = at<float>(ws, L.xs);
+    a.xs_s = c.E_s ? at<float>(ws, L.hs) : a.xs_r;
+    a.actq_r = at<void>(ws, L.actq_r); a.actq_s = c.E_s ? at<void>(ws, L.actq_s) : a.actq_r;
+    a.as_r = at<float>(ws, L.as_r); a.as_s = c.E_s ? at<float>(ws, L.as_s) : a.as_r;
+  }
   MOE_CHECK(run_ffn(c, a, offsets, (int)L.R, st, 3));
   mark_phase(5, st);
   // a8: fixed-order combine with the residual
   moe::launch_combine(h, a.out_r, c.E_s ? a.out_s : nullptr, row_of, y, c.T, c.d_model, c.K, c.E_s,
-                      c.add_residual, c.dtype, (int)L.R, st);
+                      c.add_residual, act_dtype(c.dtype), (int)L.R, st);
   mark_phase(6, st);
   // a9: the bias step, after this batch's loads are counted
   if (update_bias || max_vio_out)
@@ -475,6 +544,29 @@ moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* 
   moe::launch_router_stats(s, z, idx, kept, c.T, c.E_r, c.K, S, seq_len > 0, alpha_aux, c_z,
                            alpha_seq, rowsum, lse2, seq_counts, pchunk, stats,
                            static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
+moe_status moe_quantized_bytes(int64_t n_rows, int32_t cols, size_t* bytes) {
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows=%lld < 0", (long long)n_rows);
+  if (cols < 16 || cols % 16) return fail(MOE_ERR_INVALID_ARG, "cols=%d must be a positive multiple of 16", cols);
+  *bytes = (size_t)n_rows * cols + (size_t)n_rows * 4;
+  return MOE_OK;
+}
+
+moe_status moe_quantize_rows(const void* src, int32_t src_dtype, int64_t n_rows, int32_t cols, void* dst,
+                             void* stream) {
+  size_t unused = 0;
+  MOE_CHECK(moe_quantized_bytes(n_rows, cols, &unused));
+  if (src_dtype != MOE_DTYPE_F32 && src_dtype != MOE_DTYPE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "src_dtype=%d", src_dtype);
+  MOE_NONNULL(src); MOE_NONNULL(dst);
+  if (n_rows == 0) return MOE_OK;
+  uint8_t* codes = static_cast<uint8_t*>(dst);
+  moe::launch_quantize_rows(src, src_dtype, nullptr, 0, nullptr, n_rows, cols, codes,
+                            reinterpret_cast<float*>(codes + (size_t)n_rows * cols), nullptr,
+                            static_cast<cudaStream_t>(stream));
   return cuda_status();
 }
 

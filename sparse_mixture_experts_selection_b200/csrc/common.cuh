@@ -132,6 +132,14 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator,
 // both operands K-major, shape M x N (M = 128, N multiple of 16 up to 256).
+// Instruction descriptor of kind::f8f6f4 with e4m3 A and B (format code 0)
+// and an fp32 accumulator, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) |                       // D format: f32
+         ((uint32_t)(N >> 3) << 17) |      // N / 8
+         ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) |                       // D format: f32
          (1u << 7) |                       // A format: bf16
@@ -165,6 +173,17 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// D (+)= A * B^T with e4m3 A and B (kind::f8f6f4; 32 elements of K per
+// instruction, the same 32 bytes of each 128-byte row as the bf16 form).
+__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 

@@ -57,6 +57,7 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
 constexpr size_t SMEM_BYTES = (size_t)STAGES * (STAGE_BYTES + T_BYTES) + 1024 + 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC_Q8 = idesc_e4m3_f32(BM, BN);
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1, EPI_ROUTER = 2 };
@@ -84,6 +85,13 @@ struct Params {
   // dynamic schedule: units are claimed from this zeroed counter (null: static
   // round-robin over the CTAs)
   int* tile_counter;
+  // k-block length in elements: 64 bf16 or, with e4m3 operands (kernel
+  // template Q8), 128 e4m3 -- 128 bytes either way; for e4m3, one power-of-two
+  // scale per A row (xs) and per weight row (s0: gate or W_down, s1: up),
+  // applied to the fp32 accumulators in the epilogue
+  int bk;
+  const float *xs_r, *xs_s;
+  const float *s0_r, *s1_r, *s0_s, *s1_s;
 };
 
 constexpr int UNIT_RING = 4;     // units handed from the producer to the MMA / epilogue warps
@@ -142,7 +150,7 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
   w.mt = local % runits;
   w.nt = local / runits;
   w.kb0 = 0;
-  w.nk = ((w.sh ? p.k_s : p.k_r) + BK - 1) / BK;
+  w.nk = ((w.sh ? p.k_s : p.k_r) + p.bk - 1) / p.bk;
   const int mtiles = (w.rows + BM - 1) / BM;
   w.tail = (runits < mtiles && w.mt == runits - 1) ? w.rows - (mtiles - 1) * BM : 0;
   w.t16 = (w.tail + 15) & ~15;
@@ -158,6 +166,13 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int* 
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > kWaitLimitNs) { set_device_error(err, MOE_DEVERR_WAIT_TIMEOUT); return; }
   }
+}
+
+// One MMA of a k-step: 16 bf16 or 32 e4m3 elements of K (32 bytes of each row).
+template <bool Q8>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (Q8) tc_mma_e4m3(d, a, b, idesc, acc);
+  else tc_mma_bf16(d, a, b, idesc, acc);
 }
 
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
@@ -196,7 +211,7 @@ __device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Un
     const int e = w.sh ? w.g - p.E_r : w.g;
     c.ay = ((EPI == EPI_SWIGLU && w.sh) ? 0 : __ldg(p.grp_row0 + w.g)) + w.mt * BM;
     brow = e * (w.sh ? p.wrows_s : p.wrows_r) + w.nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
-    c.ax = c.bx = (w.kb0 + i) * BK;
+    c.ax = c.bx = (w.kb0 + i) * p.bk;
     c.by = brow;
   }
   return c;
@@ -208,8 +223,18 @@ __device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Un
 // out0 points at output row row0.
 template <int EPI>
 __device__ __forceinline__ void epilogue_transposed(const Params& p, bool sh, uint16_t* out0, size_t row0,
-                                                    int rv, int n16, int colA, int ncols, uint32_t tb) {
+                                                    int rv, int n16, int colA, int ncols, uint32_t tb,
+                                                    const float* xs, const float* wsA, const float* wsB) {
+  // e4m3 operands: xs = scales of the tile's rows (row t at xs[t]); wsA = scales
+  // of the expert's weight rows (gate, or W_down), wsB = up's (EPI_SWIGLU);
+  // xs null: bf16 operands, no scaling
   const int colB = colA + BN / 2;                     // EPI_SCALE only
+  float cA = 1.0f, cB = 1.0f;
+  if (xs && colA < ncols) {
+    cA = __ldg(wsA + colA);
+    if (EPI == EPI_SWIGLU) cB = __ldg(wsB + colA);
+  }
+  if (EPI == EPI_SCALE && xs && colB < ncols) cB = __ldg(wsA + colB);
 #pragma unroll 1
   for (int c = 0; c < n16; c += 32) {
     float dv0[32], dv1[32];
@@ -220,19 +245,23 @@ __device__ __forceinline__ void epilogue_transposed(const Params& p, bool sh, ui
       const int t = c + v;
       if (t < rv) {
         uint16_t* orow_p = out0 + (size_t)t * ncols;
+        const float rs = xs ? __ldg(xs + t) : 1.0f;
         if (EPI == EPI_SWIGLU) {
-          if (colA < ncols) orow_p[colA] = bf16_bits(silu(dv0[v]) * dv1[v]);
+          if (colA < ncols) orow_p[colA] = bf16_bits(silu(dv0[v] * (rs * cA)) * (dv1[v] * (rs * cB)));
         } else {
           const float sc = (!sh && p.row_scale) ? __ldg(p.row_scale + row0 + t) : 1.0f;
-          if (colA < ncols) orow_p[colA] = bf16_bits(dv0[v] * sc);
-          if (colB < ncols) orow_p[colB] = bf16_bits(dv1[v] * sc);
+          if (colA < ncols) orow_p[colA] = bf16_bits(dv0[v] * (rs * cA) * sc);
+          if (colB < ncols) orow_p[colB] = bf16_bits(dv1[v] * (rs * cB) * sc);
         }
       }
     }
   }
 }
 
-template <int EPI>
+// Q8: e4m3 operands (kind::f8f6f4, epilogue scales); a template parameter so
+// that the MMA issue loop carries no branch between the two MMA forms (a
+// runtime choice there cost the bf16 kernel 15 % of its throughput).
+template <int EPI, bool Q8>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -347,8 +376,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         // transposed tile: two M = 128 halves of the weight tile (gate | up, or
         // the two 128-row halves of W_down's 256) against the N = n16 rows,
         // into accumulator columns [0, n16) and [128, 128 + n16)
-        const uint32_t idesc_t = idesc_bf16_f32(BM, w.n16 ? w.n16 : 16);
-        const uint32_t idesc_tail = idesc_bf16_f32(BM, w.t16 ? w.t16 : 16);
+        constexpr bool q8 = EPI != EPI_ROUTER && Q8;
+        const uint32_t idesc_n = q8 ? IDESC_Q8 : IDESC;
+        const uint32_t idesc_t = q8 ? idesc_e4m3_f32(BM, w.n16 ? w.n16 : 16) : idesc_bf16_f32(BM, w.n16 ? w.n16 : 16);
+        const uint32_t idesc_tail = q8 ? idesc_e4m3_f32(BM, w.t16 ? w.t16 : 16) : idesc_bf16_f32(BM, w.t16 ? w.t16 : 16);
         // a unit with a merged tail holds buffer 0 (full tile) and buffer 1 (tail)
         const bool two = w.tail > 0;
         const int acc = two ? 0 : nb;
@@ -371,16 +402,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           if (w.n16 == 0) {
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
-              tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2),
-                          sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), IDESC, (kb | k) != 0);
+              tc_mma<q8>(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2),
+                     sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), idesc_n, (kb | k) != 0);
             }
           } else {
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
               const uint64_t xd = sdesc_kmajor_sw128(a0 + k * UMMA_K * 2);
-              tc_mma_bf16(d_tmem, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_t, (kb | k) != 0);
-              tc_mma_bf16(d_tmem + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
-                          idesc_t, (kb | k) != 0);
+              tc_mma<q8>(d_tmem, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_t, (kb | k) != 0);
+              tc_mma<q8>(d_tmem + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
+                     idesc_t, (kb | k) != 0);
             }
           }
           if (two) {
@@ -388,9 +419,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
               const uint64_t xd = sdesc_kmajor_sw128(t0 + k * UMMA_K * 2);
-              tc_mma_bf16(d_tail, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_tail, (kb | k) != 0);
-              tc_mma_bf16(d_tail + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
-                          idesc_tail, (kb | k) != 0);
+              tc_mma<q8>(d_tail, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), xd, idesc_tail, (kb | k) != 0);
+              tc_mma<q8>(d_tail + BN / 2, sdesc_kmajor_sw128(b0 + B_BYTES / 2 + k * UMMA_K * 2), xd,
+                     idesc_tail, (kb | k) != 0);
             }
           }
           tc_commit(&empty[stage]);       // frees the stage once these MMAs are done
@@ -438,8 +469,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       const int colA = EPI == EPI_SWIGLU ? nt * (BN / 2) + r : nt * BN + r;
       const size_t row0 = orow - r;                       // output row of the tile's row 0
       uint16_t* out0 = (sh ? p.out_s : p.out_r) + row0 * ncols;
+      // e4m3 operands: scales of the tile's A rows (xs[0] = tile row 0) and of
+      // the expert's weight rows (wsA: gate or W_down, wsB: up)
+      const float* xs = nullptr;
+      const float* wsA = nullptr;
+      const float* wsB = nullptr;
+      if (EPI != EPI_ROUTER && Q8) {
+        const int e = sh ? w.g - p.E_r : w.g;
+        const size_t wr = (size_t)e * (sh ? p.wrows_s : p.wrows_r);
+        wsA = (sh ? p.s0_s : p.s0_r) + wr;
+        wsB = (sh ? p.s1_s : p.s1_r) + wr;
+        xs = (sh ? p.xs_s : p.xs_r) + ((EPI == EPI_SWIGLU && sh) ? (size_t)mt * BM : row0);
+      }
       if (EPI != EPI_ROUTER && w.n16) {
-        epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb);
+        epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb,
+                                 xs, wsA, wsB);
       } else if (EPI == EPI_ROUTER) {
         // fp32 partial logits of split (nt % ks) for experts of column tile nt / ks
         const int ks = nt % p.r_ks, ct = nt / p.r_ks;
@@ -458,12 +502,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           }
         }
       } else if (EPI == EPI_SWIGLU) {
+        const float rs = (xs && valid) ? __ldg(xs + r) : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           float gv[32], uv[32];
           tmem_ld32(tb + c, gv);
           tmem_ld32(tb + BN / 2 + c, uv);
           const int col0 = nt * (BN / 2) + c;
+          if (xs && valid) {
+#pragma unroll
+            for (int v = 0; v < 32; ++v) {
+              const bool in = col0 + v < ncols;
+              gv[v] *= rs * (in ? __ldg(wsA + col0 + v) : 0.0f);
+              uv[v] *= rs * (in ? __ldg(wsB + col0 + v) : 0.0f);
+            }
+          }
           if (valid) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -480,11 +533,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         }
       } else {
         const float scale = (!sh && p.row_scale && valid) ? __ldg(p.row_scale + orow) : 1.0f;
+        const float rs = (xs && valid) ? __ldg(xs + r) : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float dv[32];
           tmem_ld32(tb + c, dv);
           const int col0 = nt * BN + c;
+          if (xs && valid) {
+#pragma unroll
+            for (int v = 0; v < 32; ++v) dv[v] *= rs * (col0 + v < ncols ? __ldg(wsA + col0 + v) : 0.0f);
+          }
           if (valid) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -508,7 +566,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         ph_f ^= 2u;
         tc_fence_after();
         epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
-                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN);
+                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
+                                 xs ? xs + BM : nullptr, wsA, wsB);
         tc_fence_before();
         mbar_arrive(&acc_empty[1]);
       }
@@ -541,18 +600,26 @@ static EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 matrix [rows, cols] row-major (cols contiguous), box = 64 cols x box_rows
-static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// Matrix [rows, cols] row-major (cols contiguous) of bf16 (q8 = false) or e4m3
+// bytes (q8 = true); box = one 128-byte row segment (64 bf16 / 128 e4m3) x box_rows
+static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      bool q8 = false) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint64_t strides[1] = {cols * (q8 ? 1 : 2)};
+  cuuint32_t box[2] = {(cuuint32_t)(q8 ? 2 * BK : BK), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, q8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Row scales of an e4m3 weight blob: n*rows*cols code bytes, then n*rows fp32.
+static const float* blob_scales(const void* blob, uint64_t rows, uint64_t cols) {
+  return reinterpret_cast<const float*>(static_cast<const uint8_t*>(blob) + rows * cols);
 }
 
 }  // namespace tc
@@ -610,7 +677,7 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_ROUTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_ROUTER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     attr_done[dev] = true;
   }
   const size_t n = (size_t)E * d;
@@ -633,11 +700,12 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   p.r_ks = ks; p.r_per = per;
   p.r_nkd = (d + BK - 1) / BK;
   p.zpart = zpart;
+  p.bk = BK;
   p.G = 1; p.E_r = 1;
   p.err = err;
   const int units = p.r_mtiles * p.r_ntiles * ks;
   const int grid = std::min(units, num_sms());
-  grouped_gemm_kernel<EPI_ROUTER><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  grouped_gemm_kernel<EPI_ROUTER, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
   *ks_out = ks;
   return cudaGetLastError();
 }
@@ -648,11 +716,14 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     attr_done[dev] = true;
   }
   const bool has_s = a.E_s > 0;
+  const bool q8 = a.q8 != 0;
   Params p{};
   bool ok = true;
   p.grp_rows = a.grp_rows;
@@ -660,18 +731,25 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   p.G = a.E_r + a.E_s;
   p.E_r = a.E_r;
   p.err = a.err;
+  p.bk = q8 ? 2 * BK : BK;
   if (which == 0) {
     // gate/up: A = permuted tokens (routed) or h (shared); B = gate | up, 128 rows each
     const uint64_t wr_r = (uint64_t)a.E_r * a.f_r, wr_s = has_s ? (uint64_t)a.E_s * a.f_s : wr_r;
-    ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM);
-    ok &= make_tmap(&p.a_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d, BM);
-    ok &= make_tmap(&p.a32_r, a.x_r, (uint64_t)a.max_rows_r, a.d, A_SUB_ROWS);
+    ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM, q8);
+    ok &= make_tmap(&p.a_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d, BM, q8);
+    ok &= make_tmap(&p.a32_r, a.x_r, (uint64_t)a.max_rows_r, a.d, A_SUB_ROWS, q8);
     ok &= make_tmap(&p.a32_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d,
-                    A_SUB_ROWS);
-    ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, BN / 2);
-    ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, BN / 2);
-    ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, BN / 2);
-    ok &= make_tmap(&p.b1_s, has_s ? a.wu_s : a.wu_r, wr_s, a.d, BN / 2);
+                    A_SUB_ROWS, q8);
+    ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, BN / 2, q8);
+    ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, BN / 2, q8);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, BN / 2, q8);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wu_s : a.wu_r, wr_s, a.d, BN / 2, q8);
+    if (q8) {
+      p.xs_r = a.xs_r; p.xs_s = has_s ? a.xs_s : a.xs_r;
+      p.s0_r = blob_scales(a.wg_r, wr_r, a.d); p.s1_r = blob_scales(a.wu_r, wr_r, a.d);
+      p.s0_s = has_s ? blob_scales(a.wg_s, wr_s, a.d) : p.s0_r;
+      p.s1_s = has_s ? blob_scales(a.wu_s, wr_s, a.d) : p.s1_r;
+    }
     p.prefix = a.pre_gu;
     p.k_r = p.k_s = a.d;
     p.wrows_r = a.f_r; p.wrows_s = a.f_s;
@@ -683,14 +761,22 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
     const uint64_t rows_s = has_s ? (uint64_t)a.E_s * a.T : (uint64_t)a.max_rows_r;
     const int fs = has_s ? a.f_s : a.f_r;
     const uint64_t wd_rows_s = (uint64_t)(has_s ? a.E_s : a.E_r) * a.d;
-    ok &= make_tmap(&p.a_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, BM);
-    ok &= make_tmap(&p.a_s, has_s ? a.act_s : a.act_r, rows_s, fs, BM);
-    ok &= make_tmap(&p.a32_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, A_SUB_ROWS);
-    ok &= make_tmap(&p.a32_s, has_s ? a.act_s : a.act_r, rows_s, fs, A_SUB_ROWS);
-    ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
-    ok &= make_tmap(&p.b1_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN);
-    ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN);
-    ok &= make_tmap(&p.b1_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN);
+    // e4m3: the down GEMM reads the quantized copy of A (act_q) and its row scales
+    const void* A_r = q8 ? a.actq_r : a.act_r;
+    const void* A_s = q8 ? a.actq_s : a.act_s;
+    ok &= make_tmap(&p.a_r, A_r, (uint64_t)a.max_rows_r, a.f_r, BM, q8);
+    ok &= make_tmap(&p.a_s, has_s ? A_s : A_r, rows_s, fs, BM, q8);
+    ok &= make_tmap(&p.a32_r, A_r, (uint64_t)a.max_rows_r, a.f_r, A_SUB_ROWS, q8);
+    ok &= make_tmap(&p.a32_s, has_s ? A_s : A_r, rows_s, fs, A_SUB_ROWS, q8);
+    ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN, q8);
+    ok &= make_tmap(&p.b1_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BN, q8);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN, q8);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, BN, q8);
+    if (q8) {
+      p.xs_r = a.as_r; p.xs_s = has_s ? a.as_s : a.as_r;
+      p.s0_r = p.s1_r = blob_scales(a.wd_r, (uint64_t)a.E_r * a.d, a.f_r);
+      p.s0_s = p.s1_s = has_s ? blob_scales(a.wd_s, wd_rows_s, fs) : p.s0_r;
+    }
     p.prefix = a.pre_dn;
     p.k_r = a.f_r; p.k_s = a.f_s;
     p.wrows_r = a.d; p.wrows_s = a.d;
@@ -701,10 +787,14 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   if (!ok) return cudaErrorInvalidValue;
   p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
   const int grid = num_sms();
-  if (which == 0)
-    grouped_gemm_kernel<EPI_SWIGLU><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  if (which == 0 && q8)
+    grouped_gemm_kernel<EPI_SWIGLU, true><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  else if (which == 0)
+    grouped_gemm_kernel<EPI_SWIGLU, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  else if (q8)
+    grouped_gemm_kernel<EPI_SCALE, true><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
   else
-    grouped_gemm_kernel<EPI_SCALE><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+    grouped_gemm_kernel<EPI_SCALE, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
   return cudaGetLastError();
 }
 

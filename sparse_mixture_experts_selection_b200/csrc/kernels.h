@@ -18,6 +18,14 @@ struct FfnArgs {
   void *act_r, *act_s, *out_r, *out_s;
   int* err;
   int* tile_counters;   // [2] unit counters of the two GEMMs, zeroed by groups_kernel
+  // e4m3 expert weights (q8 = 1): x_r / x_s and the weights are e4m3 codes
+  // (weights: blobs of codes followed by fp32 row scales), xs_r / xs_s the row
+  // scales of x; the SwiGLU output act_* (bf16) is quantized into actq_* with
+  // row scales as_* before the down GEMM
+  int q8;
+  const float *xs_r, *xs_s;
+  void *actq_r, *actq_s;
+  float *as_r, *as_s;
 };
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
@@ -51,6 +59,14 @@ void launch_router_stats(const float* s, const float* z, const int32_t* idx, con
                          int T, int E, int K, int seq_len, int use_seq, float alpha_aux, float c_z,
                          float alpha_seq, float* rowsum, float* lse2, int* seq_counts, float* pseq,
                          float* stats, cudaStream_t st);
+
+// e4m3 rows with one power-of-two scale per row (src_dtype 1 = bf16, else fp32;
+// cols a multiple of 16).  Row r reads source row src_row[r] (< n_src) when
+// src_row is given, else row r; rows at or beyond *n_rows_ptr (when given) are
+// skipped.
+void launch_quantize_rows(const void* src, int src_dtype, const int32_t* src_row, int n_src,
+                          const int* n_rows_ptr, int64_t n_rows, int cols, uint8_t* codes,
+                          float* scales, int* err, cudaStream_t st);
 
 int simt_bm();
 int simt_bn();

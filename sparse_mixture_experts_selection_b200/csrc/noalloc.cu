@@ -95,6 +95,6 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                       row_gate, err, s);
   if (x_perm)
     moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model,
-                       c.dtype == MOE_DTYPE_BF16 ? 2 : 4, c.T * c.K, c.T, err, s);
+                       c.dtype == MOE_DTYPE_F32 ? 4 : 2, c.T * c.K, c.T, err, s);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

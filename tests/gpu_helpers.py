@@ -22,7 +22,7 @@ F32_TOL = 1e-4    # ... for fp32 layers
 
 
 def torch_dtype(w):
-    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    return torch.bfloat16 if w.dtype != "f32" else torch.float32
 
 
 def to_dev(x: np.ndarray, dtype=torch.float32):
@@ -74,7 +74,7 @@ class LazyHostWeights:
 def device_weights(w):
     """All weights of a workload generated directly on the device (CUDA twin)."""
     dt = torch_dtype(w)
-    bf16 = w.dtype == "bf16"
+    bf16 = w.dtype != "f32"
     out = {}
     for k in ("gate", "up", "down", "sgate", "sup", "sdown"):
         tid, n, rows, cols, sigma = mi.weight_spec(w, k)
@@ -151,4 +151,4 @@ def check_close(y_gpu: np.ndarray, y_ref: np.ndarray, h: np.ndarray, tol: float,
 
 
 def out_eps_of(w) -> float:
-    return 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -22
+    return 2.0 ** -8 if w.dtype != "f32" else 2.0 ** -22

@@ -45,7 +45,7 @@ SMALL = {
 
 
 def tol_of(w):
-    return BF16_TOL if w.dtype == "bf16" else F32_TOL
+    return BF16_TOL if w.dtype != "f32" else F32_TOL
 
 
 def inputs(w, step=0):

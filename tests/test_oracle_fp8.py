@@ -53,6 +53,9 @@ def test_pow2_scale_closed_form():
     assert np.all(a / s <= 448.0) and np.all(a / (s / 2) > 448.0)             # smallest such
     edge = np.array([448.0, np.nextafter(F32(448.0), F32(1e9)), 0.0, 1.0, 1.75, 1.7500001, 224.0], F32)
     assert list(mo.pow2_scale(edge)) == [1.0, 2.0, 1.0, 2.0 ** -8, 2.0 ** -8, 2.0 ** -7, 0.5]
+    # the scale stays a normal fp32 number for tiny rows
+    tiny = np.array([2.0 ** -120, 2.0 ** -140, np.finfo(F32).smallest_subnormal], F32)
+    assert list(mo.pow2_scale(tiny)) == [2.0 ** -126] * 3
 
 
 def test_quantize_rows_error_bound():
