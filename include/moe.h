@@ -262,8 +262,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
  *   are not used by this call).  Deterministic (no floating-point atomics).
  */
 /*
- * Expert weights in fewer bits ("GPUs, memory and failures", serving notes:
- * storing weights in fewer bits for the weight-streaming regime; the pages
+ * Low-precision expert weights ("GPUs, memory and failures", serving notes:
+ * lower-precision expert weights when serving is bound by streaming them; the pages
  * fix no format -- this is the library's): e4m3 codes with one power-of-two
  * scale per row, the smallest s with max_c |x[r][c]| / s <= 448 (at least
  * 2^-126; 1 for an all-zero row), each element x / s rounded to the nearest

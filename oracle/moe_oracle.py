@@ -400,8 +400,8 @@ def dropped_rate(kept: np.ndarray, counts: np.ndarray) -> float:
 
 
 # ---------------------------------------------------------------------------
-# Expert weights in fewer bits ([GMF], "storing weights in fewer bits" for the
-# weight-streaming regime).  The pages name no format; the reading here (also
+# Low-precision expert weights ([GMF] suggests keeping expert weights at lower
+# precision when serving is bound by streaming them).  The pages name no format; the reading here (also
 # in the design notes): fp8 e4m3 codes (1 sign, 4 exponent bits with bias 7,
 # 3 mantissa bits, no infinities, largest finite 448) with one power-of-two
 # scale per weight row (output channel) and per activation row (token); the

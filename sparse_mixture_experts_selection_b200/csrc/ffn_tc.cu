@@ -7,8 +7,8 @@
 //
 // SwiGLU(h) = (SiLU(h W_gate^T) * (h W_up^T)) W_down^T and the gate-weighted
 // routed sum follow "Sparse Mixture-of-Experts (MoE): Routing Math, Load
-// Balancing & Expert Parallelism" (section 0 layer equation; section 3 "a
-// single fused Grouped GEMM over variable-sized token buckets").
+// Balancing & Expert Parallelism" (section 0 layer equation; section 3: all
+// local experts run as one grouped GEMM over their variable-length row groups).
 //
 // Work unit = (group, 128-row tile, 256-column B tile).  Groups are the routed
 // experts (expert-contiguous rows of the permuted activations) followed by the

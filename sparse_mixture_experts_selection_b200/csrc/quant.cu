@@ -1,13 +1,13 @@
-// e4m3 quantization of matrix rows (expert weights in fewer bits, and the rows
+// e4m3 quantization of matrix rows (low-precision expert weights, and the rows
 // entering the e4m3 GEMMs): one power-of-two scale per row, the smallest s with
 // amax / s <= 448, then each element x / s rounded to the nearest e4m3 value
 // (ties to the even code, saturating at 448).  Dividing by a power of two is
 // exact, so the codes depend only on the row's values -- no division rounding
 // and no dependence on how amax was reduced.
 //
-// "Storing weights in fewer bits" for the weight-streaming regime is named by
-// "GPUs, memory and failures" (serving notes); the pages fix no format, so
-// the per-row power-of-two e4m3 layout is this library's reading.
+// "GPUs, memory and failures" (serving notes) suggests lower-precision expert
+// weights when serving is bound by streaming them; the pages fix no format,
+// so the per-row power-of-two e4m3 layout is this library's reading.
 #include <cuda_fp8.h>
 
 #include "common.cuh"

@@ -1,4 +1,4 @@
-"""Pins of the oracle's e4m3 quantization (expert weights in fewer bits):
+"""Pins of the oracle's e4m3 quantization (low-precision expert weights):
 the e4m3 format's landmarks, torch's own float8_e4m3fn conversion, ties to
 even at every midpoint, saturation, the closed form of the power-of-two row
 scale, the per-element error bound, and the quantized expert against the
