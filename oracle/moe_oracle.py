@@ -60,6 +60,10 @@ quantize_rows, swiglu_q8, layer_output_q8) is pinned in
 tests/test_oracle_fp8.py against torch's float8_e4m3fn conversion, ties to
 even, the closed form of the scale and the format's error bound; the
 quantized expert's values beyond that bound are "parity unpinned".
+The layer backward (swiglu_backward, gate_backward, score_backward,
+layer_backward) is pinned in tests/test_oracle_backward.py against
+torch.autograd through a dense restatement of the forward, finite
+differences, and planted mistakes.
 """
 from __future__ import annotations
 
@@ -502,3 +506,87 @@ def layer_output_q8(cfg: LayerConfig, h: np.ndarray, idx: np.ndarray, gates: np.
         o = swiglu_q8(x[rows], weights("gate", ex), weights("up", ex), weights("down", ex))
         y[rows] += gates[tok[rows], ks].astype(np.float64)[:, None] * o
     return y
+
+
+# ---------------------------------------------------------------------------
+# Backward pass of the layer ([SMoE] section 2: the selection uses s + b but
+# the gates g are built from s alone, so the gradient reaches the router
+# through g and never reaches the bias; [EPLB]: the bias is a buffer updated
+# by the sign rule, not by gradient descent).  The selected set I_t and the
+# capacity decisions are piecewise constant: no gradient flows through them.
+# Everything in float64.
+# ---------------------------------------------------------------------------
+
+def swiglu_backward(x, w_gate, w_up, w_down, d_out):
+    """Gradients of one SwiGLU expert o = (SiLU(x Wg^T) * (x Wu^T)) Wd^T for
+    rows x [n, d] and the output gradient d_out [n, d]:
+    (dx, dWg, dWu, dWd, o) -- o is returned for the gate gradient."""
+    x = np.asarray(x, np.float64)
+    wg, wu, wd = (np.asarray(w, np.float64) for w in (w_gate, w_up, w_down))
+    do = np.asarray(d_out, np.float64)
+    u = x @ wg.T
+    v = x @ wu.T
+    sig = 1.0 / (1.0 + np.exp(-u))
+    a = u * sig * v
+    da = do @ wd                                   # dL/da  [n, f]
+    du = da * v * sig * (1.0 + u * (1.0 - sig))    # SiLU'(u) = sig (1 + u (1 - sig))
+    dv = da * u * sig
+    dx = du @ wg + dv @ wu
+    return dx, du.T @ x, dv.T @ x, do.T @ a, a @ wd.T
+
+
+def gate_backward(s32: np.ndarray, idx: np.ndarray, dg: np.ndarray) -> np.ndarray:
+    """dL/ds [T, E] from dL/dg [T, K] with g_k = s_{I_k} / max(S, 1e-12),
+    S = sum_k s_{I_k}: ds_j = (dg_j - sum_k g_k dg_k) / S for j in I_t (the
+    clamp inactive), ds_j = dg_j / 1e-12 when it is active, 0 outside I_t."""
+    s = np.asarray(s32, np.float64)
+    T = s.shape[0]
+    sel = np.take_along_axis(s, idx.astype(np.int64), axis=1)
+    S = sel.sum(axis=1)
+    den = np.maximum(S, float(GATE_EPS))
+    g = sel / den[:, None]
+    dg = np.asarray(dg, np.float64)
+    corr = np.where(S > float(GATE_EPS), (g * dg).sum(axis=1), 0.0)
+    ds = np.zeros_like(s)
+    np.put_along_axis(ds, idx.astype(np.int64), (dg - corr[:, None]) / den[:, None], axis=1)
+    return ds
+
+
+def score_backward(s32: np.ndarray, ds: np.ndarray, score_fn: int) -> np.ndarray:
+    """dL/dz from dL/ds: sigmoid s(1 - s); softmax p * (ds - <ds, p>)."""
+    s = np.asarray(s32, np.float64)
+    if score_fn == 0:
+        return ds * s * (1.0 - s)
+    return s * (ds - (ds * s).sum(axis=1, keepdims=True))
+
+
+def layer_backward(cfg: LayerConfig, h: np.ndarray, e: np.ndarray, s32: np.ndarray,
+                   idx: np.ndarray, gates: np.ndarray, disp: Dispatch, weights: WeightSource,
+                   dy: np.ndarray):
+    """Gradients of the layer output y w.r.t. h, the centroids e and every
+    expert weight, for the routing (idx, gates, disp) of the forward pass and
+    dL/dy.  Returns dict(dh, de, dg, grads) with grads[(which, expert)]."""
+    x = np.asarray(h, np.float64)
+    dy = np.asarray(dy, np.float64)
+    dh = dy * float(cfg.add_residual)
+    grads = {}
+    for j in range(cfg.E_s):
+        dx, dwg, dwu, dwd, _ = swiglu_backward(x, weights("sgate", j), weights("sup", j),
+                                               weights("sdown", j), dy)
+        dh = dh + dx
+        grads[("sgate", j)], grads[("sup", j)], grads[("sdown", j)] = dwg, dwu, dwd
+    dg = np.zeros((cfg.T, cfg.K))
+    kept = disp.row_of >= 0
+    ex_of = idx.astype(np.int64)
+    for ex in np.unique(ex_of[kept]):
+        rows, ks = np.nonzero((ex_of == ex) & kept)
+        g = gates[rows, ks].astype(np.float64)[:, None]
+        dx, dwg, dwu, dwd, o = swiglu_backward(x[rows], weights("gate", ex), weights("up", ex),
+                                               weights("down", ex), g * dy[rows])
+        np.add.at(dh, rows, dx)
+        dg[rows, ks] = (dy[rows] * o).sum(axis=1)
+        grads[("gate", ex)], grads[("up", ex)], grads[("down", ex)] = dwg, dwu, dwd
+    dz = score_backward(s32, gate_backward(s32, idx, dg), cfg.score_fn)
+    dh = dh + dz @ np.asarray(e, np.float64)
+    de = dz.T @ x
+    return dict(dh=dh, de=de, dg=dg, dz=dz, grads=grads)
