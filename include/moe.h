@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum {
   MOE_OK = 0,
@@ -110,6 +110,9 @@ typedef struct {
   float capacity_factor; /* <= 0: dropless; else C = floor(T*K*CF/E_r) rows per expert  */
   int32_t dtype;         /* MOE_DTYPE_F32, MOE_DTYPE_BF16 or MOE_DTYPE_BF16_E4M3         */
   int32_t add_residual;  /* 1: y includes h_t                                           */
+  int32_t train;         /* 1: moe_layer_forward keeps what moe_layer_backward needs in
+                            the workspace (bf16 layers; d_model, d_ffn, d_ffn_shared
+                            multiples of 64); 0: inference                             */
 } moe_config;
 
 /* Library ABI version (MOE_ABI_VERSION). */
@@ -261,6 +264,34 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
  *   ws: at least moe_router_stats_workspace_size bytes (its first 256 bytes
  *   are not used by this call).  Deterministic (no floating-point atomics).
  */
+/*
+ * Backward of moe_layer_forward (train = 1): gradients of a loss L, given
+ * dy = dL/dy [T, d] (bf16), with respect to h, the centroids e and every
+ * expert weight, for the routing the forward chose.  The derivative of the
+ * layer equation ("Sparse Mixture-of-Experts ...", section 0) per expert,
+ * through the gates g = s / sum_{I_t} s (section 2: the selection uses s + b,
+ * the gates s alone, so no gradient reaches the bias b, and the top-K choice
+ * and capacity drops are held fixed).
+ *
+ *   h, e, weights: the forward's inputs; s [T, E_r] fp32 and idx [T, K] the
+ *   scores and selections the forward exported (s_out, idx_out).
+ *   ws: the workspace of the forward call just before, with the same cfg
+ *   (train = 1) -- it still holds the permutation, x, U | V, A and the
+ *   slots; this call overwrites its group tables.
+ *   Outputs: dh [T, d] bf16 (residual + shared + routed + router terms, summed
+ *   in fp32 in a fixed order); de [E_r, d] fp32; dW_gate, dW_up [E_r, f, d],
+ *   dW_down [E_r, d, f] bf16 (zero for experts without kept rows); the shared
+ *   experts' dWs_* likewise (NULL when E_s = 0).
+ *   Deterministic (no floating-point atomics).
+ */
+moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float* e, const float* s,
+                              const int32_t* idx, const void* w_gate, const void* w_up,
+                              const void* w_down, const void* ws_gate, const void* ws_up,
+                              const void* ws_down, const void* dy, void* dh, float* de,
+                              void* dw_gate, void* dw_up, void* dw_down, void* dws_gate,
+                              void* dws_up, void* dws_down, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /*
  * Low-precision expert weights ("GPUs, memory and failures", serving notes:
  * lower-precision expert weights when serving is bound by streaming them; the pages

@@ -22,7 +22,7 @@ __all__ = [
     "moe_expert_ffn", "moe_expert_ffn_workspace_size", "moe_combine", "moe_bias_update",
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
     "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
-    "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3",
+    "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3", "moe_layer_backward",
     "moe_set_phase_events", "moe_selftest_bounded_wait",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
@@ -40,7 +40,8 @@ class MoeConfig(ctypes.Structure):
                 ("d_ffn_shared", ctypes.c_int32), ("score_fn", ctypes.c_int32),
                 ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
                 ("group_topn", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
-                ("dtype", ctypes.c_int32), ("add_residual", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("add_residual", ctypes.c_int32),
+                ("train", ctypes.c_int32)]
 
 
 class MoeError(RuntimeError):
@@ -71,6 +72,7 @@ SIGNATURES = {
                                          ctypes.c_size_t, _P]),
     "moe_router_stats_workspace_size": (ctypes.c_int, [_P, _I32, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_quantized_bytes": (ctypes.c_int, [ctypes.c_int64, _I32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_layer_backward": (ctypes.c_int, [_P] * 20 + [_P, ctypes.c_size_t, _P]),
     "moe_quantize_rows": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _I32, _P, _P]),
     "moe_router_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
@@ -176,6 +178,15 @@ def moe_quantized_bytes(n_rows: int, cols: int) -> int:
 def moe_quantize_rows(src, src_dtype: int, n_rows: int, cols: int, dst, stream=None):
     _check(lib().moe_quantize_rows(_ptr(src), int(src_dtype), int(n_rows), int(cols), _ptr(dst),
                                    _stream(stream)))
+
+
+def moe_layer_backward(cfg, h, e, s, idx, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dy, dh, de,
+                       dw_gate, dw_up, dw_down, dws_gate, dws_up, dws_down, ws, stream=None):
+    """Gradients of the last moe_layer_forward (cfg.train = 1, same workspace)."""
+    _check(lib().moe_layer_backward(
+        ctypes.byref(cfg), _ptr(h), _ptr(e), _ptr(s), _ptr(idx), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dh), _ptr(de), _ptr(dw_gate), _ptr(dw_up),
+        _ptr(dw_down), _ptr(dws_gate), _ptr(dws_up), _ptr(dws_down), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 # order of the values moe_router_stats writes

@@ -46,6 +46,8 @@ struct Layout {
   // e4m3-weight layers: row scales of x_perm (codes), the e4m3 copy of h and its
   // scales (shared experts), the e4m3 copies of A and their scales
   size_t xs, hq, hs, actq_r, actq_s, as_r, as_s;
+  // training: U | V kept by the forward; the backward's dO, dL/dg, dz, dU | dV, dX
+  size_t uv_r, uv_s, dO, dg_row, dz, duv_r, duv_s, dx_r, dx_s;
   size_t total;
   int n_chunks;
   int64_t cap, R;
@@ -96,6 +98,17 @@ Layout make_layout(const moe_config& c) {
   L.actq_s = take(q8 ? (size_t)c.E_s * c.T * fs : 0);
   L.as_r = take(q8 ? (size_t)L.R * 4 : 0);
   L.as_s = take(q8 ? (size_t)c.E_s * c.T * 4 : 0);
+  const bool tr = c.train != 0;
+  const size_t rs = (size_t)c.E_s * c.T;
+  L.uv_r = take(tr ? (size_t)L.R * 2 * c.d_ffn * 2 : 0);
+  L.uv_s = take(tr ? rs * 2 * fs * 2 : 0);
+  L.dO = take(tr ? (size_t)L.R * c.d_model * 2 : 0);
+  L.dg_row = take(tr ? (size_t)L.R * 4 : 0);
+  L.dz = take(tr ? (size_t)c.T * c.E_r * 4 : 0);
+  L.duv_r = take(tr ? (size_t)L.R * 2 * c.d_ffn * 2 : 0);
+  L.duv_s = take(tr ? rs * 2 * fs * 2 : 0);
+  L.dx_r = take(tr ? (size_t)L.R * c.d_model * 2 : 0);
+  L.dx_s = take(tr ? rs * c.d_model * 2 : 0);
   L.total = o;
   return L;
 }
@@ -136,6 +149,10 @@ moe_status validate(const moe_config* cfg) {
     return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d_model, d_ffn, d_ffn_shared >= 64");
   if (is_q8(c.dtype) && (c.d_model % 16 || c.d_ffn % 16 || (c.E_s > 0 && c.d_ffn_shared % 16)))
     return fail(MOE_ERR_UNSUPPORTED, "e4m3 weights need d_model, d_ffn, d_ffn_shared multiples of 16");
+  if (c.train != 0 && c.train != 1) return fail(MOE_ERR_INVALID_ARG, "train=%d", c.train);
+  if (c.train && c.dtype != MOE_DTYPE_BF16) return fail(MOE_ERR_UNSUPPORTED, "train needs MOE_DTYPE_BF16");
+  if (c.train && (c.d_model % 64 || c.d_ffn % 64 || (c.E_s > 0 && c.d_ffn_shared % 64)))
+    return fail(MOE_ERR_UNSUPPORTED, "train needs d_model, d_ffn, d_ffn_shared multiples of 64");
   return MOE_OK;
 }
 
@@ -470,6 +487,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   a.out_r = at<void>(ws, L.slot_r); a.out_s = c.E_s ? at<void>(ws, L.slot_s) : a.out_r;
   a.err = err;
   a.tile_counters = err + 16;          // spare words of the error block
+  if (c.train) { a.uv_r = at<void>(ws, L.uv_r); a.uv_s = c.E_s ? at<void>(ws, L.uv_s) : a.uv_r; }
   if (q8) {
     a.q8 = 1;
     a.x_s = c.E_s ? at<void>(ws, L.hq) : x_perm;
@@ -488,6 +506,71 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   if (update_bias || max_vio_out)
     moe::launch_bias_update(counts, update_bias ? b : nullptr, gamma, max_vio_out, c.E_r, c.K, c.T, st);
   mark_phase(7, st);
+  return cuda_status();
+}
+
+moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float* e, const float* s,
+                              const int32_t* idx, const void* w_gate, const void* w_up,
+                              const void* w_down, const void* ws_gate, const void* ws_up,
+                              const void* ws_down, const void* dy, void* dh, float* de,
+                              void* dw_gate, void* dw_up, void* dw_down, void* dws_gate,
+                              void* dws_up, void* dws_down, void* ws, size_t ws_bytes, void* stream) {
+  MOE_CHECK(validate(cfg));
+  const moe_config& c = *cfg;
+  if (!c.train) return fail(MOE_ERR_INVALID_ARG, "cfg->train must be 1 (forward and backward)");
+  MOE_NONNULL(h); MOE_NONNULL4(e); MOE_NONNULL4(s); MOE_NONNULL4(idx);
+  MOE_NONNULL(w_gate); MOE_NONNULL(w_up); MOE_NONNULL(w_down);
+  MOE_NONNULL(dy); MOE_NONNULL(dh); MOE_NONNULL(de);
+  MOE_NONNULL(dw_gate); MOE_NONNULL(dw_up); MOE_NONNULL(dw_down);
+  if (c.E_s > 0) {
+    MOE_NONNULL(ws_gate); MOE_NONNULL(ws_up); MOE_NONNULL(ws_down);
+    MOE_NONNULL(dws_gate); MOE_NONNULL(dws_up); MOE_NONNULL(dws_down);
+  }
+  const Layout L = make_layout(c);
+  MOE_CHECK(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err = at<int>(ws, L.err);
+  const int* offsets = at<int>(ws, L.offsets);
+  const int fs = c.E_s ? c.d_ffn_shared : c.d_ffn;
+  const int R = (int)L.R;
+  // group tables of the backward GEMMs: plain 128-row tiles, 256-column tiles of f (dA) and d (dX)
+  moe::launch_groups(offsets, c.E_r, c.E_s, c.T, 128, 0, (c.d_ffn + 255) / 256, (fs + 255) / 256,
+                     (c.d_model + 255) / 256, (c.d_model + 255) / 256, at<int>(ws, L.grp_rows),
+                     at<int>(ws, L.grp_row0), at<int>(ws, L.pre_gu), at<int>(ws, L.pre_dn), R, err, err + 16, st);
+  moe::BwdRouteArgs ra{};
+  ra.T = c.T; ra.d = c.d_model; ra.E = c.E_r; ra.K = c.K; ra.E_s = c.E_s; ra.score_fn = c.score_fn;
+  ra.add_residual = c.add_residual; ra.max_rows = R;
+  ra.dy = static_cast<const uint16_t*>(dy); ra.slot = at<uint16_t>(ws, L.slot_r);
+  ra.dx_r = at<uint16_t>(ws, L.dx_r); ra.dx_s = at<uint16_t>(ws, L.dx_s);
+  ra.h = static_cast<const uint16_t*>(h);
+  ra.perm_tok = at<int32_t>(ws, L.perm_tok); ra.row_of = at<int32_t>(ws, L.row_of); ra.idx = idx;
+  ra.n_rows_ptr = offsets + c.E_r;
+  ra.row_gate = at<float>(ws, L.row_gate); ra.s = s; ra.e = e;
+  ra.dO = at<uint16_t>(ws, L.dO); ra.dh = static_cast<uint16_t*>(dh);
+  ra.dg_row = at<float>(ws, L.dg_row); ra.dz = at<float>(ws, L.dz); ra.de = de;
+  ra.err = err;
+  moe::launch_bwd_route(ra, st);                      // dO = g dy, dL/dg per kept row
+  moe::BwdArgs ba{};
+  ba.T = c.T; ba.d = c.d_model; ba.f_r = c.d_ffn; ba.f_s = fs; ba.E_r = c.E_r; ba.E_s = c.E_s;
+  ba.max_rows_r = R;
+  ba.dO_r = ra.dO; ba.dy = dy;
+  ba.wg_r = w_gate; ba.wu_r = w_up; ba.wd_r = w_down;
+  ba.wg_s = c.E_s ? ws_gate : w_gate; ba.wu_s = c.E_s ? ws_up : w_up; ba.wd_s = c.E_s ? ws_down : w_down;
+  ba.uv_r = at<void>(ws, L.uv_r); ba.uv_s = c.E_s ? at<void>(ws, L.uv_s) : ba.uv_r;
+  ba.duv_r = at<void>(ws, L.duv_r); ba.duv_s = c.E_s ? at<void>(ws, L.duv_s) : ba.duv_r;
+  ba.dx_r = at<void>(ws, L.dx_r); ba.dx_s = c.E_s ? at<void>(ws, L.dx_s) : ba.dx_r;
+  ba.x_r = at<void>(ws, L.x_perm); ba.h = h;
+  ba.act_r = at<void>(ws, L.act_r); ba.act_s = c.E_s ? at<void>(ws, L.act_s) : ba.act_r;
+  ba.dwg_r = dw_gate; ba.dwu_r = dw_up; ba.dwd_r = dw_down;
+  ba.dwg_s = dws_gate; ba.dwu_s = dws_up; ba.dwd_s = dws_down;
+  ba.grp_rows = at<int>(ws, L.grp_rows); ba.grp_row0 = at<int>(ws, L.grp_row0);
+  ba.pre_da = at<int>(ws, L.pre_gu); ba.pre_dx = at<int>(ws, L.pre_dn);
+  ba.err = err;
+  for (int which = 0; which < 5; ++which) {
+    cudaError_t er = moe::launch_bwd_tc(ba, which, st);
+    if (er != cudaSuccess) return fail(MOE_ERR_CUDA, "backward GEMM %d: %s", which, cudaGetErrorString(er));
+  }
+  moe::launch_bwd_gate_dh_de(ra, st);                 // dz, dh, de
   return cuda_status();
 }
 

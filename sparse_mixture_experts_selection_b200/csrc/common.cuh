@@ -130,8 +130,23 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator,
-// both operands K-major, shape M x N (M = 128, N multiple of 16 up to 256).
+// Shared-memory matrix descriptor of an MN-major operand with 128-byte swizzle,
+// as TMA writes a row-major tile loaded in boxes of {64 MN-elements, K rows}:
+// each K index is one 128-byte line of 64 MN-elements, 8 lines form a swizzle
+// atom (SBO = 1024 bytes between 8-line groups along K) and consecutive
+// 64-element MN blocks sit 8192 bytes apart (LBO; boxes of 64 K-lines).  The
+// k-th 16-element K slice starts 16 lines (2048 bytes) further.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Make this thread's generic-proxy writes to shared memory visible to later
+// async-proxy readers (the tensor core's operand fetch).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Instruction descriptor of kind::f8f6f4 with e4m3 A and B (format code 0)
 // and an fp32 accumulator, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
@@ -140,6 +155,11 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);       // M / 16
 }
 
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator,
+// both operands K-major, shape M x N (M = 128, N multiple of 16 up to 256);
+// OR in kIdescAMnMajor / kIdescBMnMajor for MN-major operands.
+constexpr uint32_t kIdescAMnMajor = 1u << 15;
+constexpr uint32_t kIdescBMnMajor = 1u << 16;
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) |                       // D format: f32
          (1u << 7) |                       // A format: bf16

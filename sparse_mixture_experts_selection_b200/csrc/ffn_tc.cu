@@ -92,6 +92,10 @@ struct Params {
   int bk;
   const float *xs_r, *xs_s;
   const float *s0_r, *s1_r, *s0_s, *s1_s;
+  // training forward (EPI_SWIGLU): the pre-activations U | V of every row,
+  // [rows, 2f] bf16 (U in columns 0..f-1, V in f..2f-1), for the backward
+  uint16_t* uv_r;
+  uint16_t* uv_s;
 };
 
 constexpr int UNIT_RING = 4;     // units handed from the producer to the MMA / epilogue warps
@@ -222,9 +226,10 @@ __device__ __forceinline__ TileCoords<EPI> tile_coords(const Params& p, const Un
 // second half, columns [128, 128 + n16)); accumulator column t = row row0 + t.
 // out0 points at output row row0.
 template <int EPI>
-__device__ __forceinline__ void epilogue_transposed(const Params& p, bool sh, uint16_t* out0, size_t row0,
+__device__ __noinline__ void epilogue_transposed(const Params& p, bool sh, uint16_t* out0, size_t row0,
                                                     int rv, int n16, int colA, int ncols, uint32_t tb,
-                                                    const float* xs, const float* wsA, const float* wsB) {
+                                                    const float* xs, const float* wsA, const float* wsB,
+                                                    uint16_t* uv0) {
   // e4m3 operands: xs = scales of the tile's rows (row t at xs[t]); wsA = scales
   // of the expert's weight rows (gate, or W_down), wsB = up's (EPI_SWIGLU);
   // xs null: bf16 operands, no scaling
@@ -247,7 +252,14 @@ __device__ __forceinline__ void epilogue_transposed(const Params& p, bool sh, ui
         uint16_t* orow_p = out0 + (size_t)t * ncols;
         const float rs = xs ? __ldg(xs + t) : 1.0f;
         if (EPI == EPI_SWIGLU) {
-          if (colA < ncols) orow_p[colA] = bf16_bits(silu(dv0[v] * (rs * cA)) * (dv1[v] * (rs * cB)));
+          if (colA < ncols) {
+            const float g = dv0[v] * (rs * cA), u = dv1[v] * (rs * cB);
+            orow_p[colA] = bf16_bits(silu(g) * u);
+            if (uv0) {
+              uv0[(size_t)t * 2 * ncols + colA] = bf16_bits(g);
+              uv0[(size_t)t * 2 * ncols + ncols + colA] = bf16_bits(u);
+            }
+          }
         } else {
           const float sc = (!sh && p.row_scale) ? __ldg(p.row_scale + row0 + t) : 1.0f;
           if (colA < ncols) orow_p[colA] = bf16_bits(dv0[v] * (rs * cA) * sc);
@@ -481,9 +493,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         wsB = (sh ? p.s1_s : p.s1_r) + wr;
         xs = (sh ? p.xs_s : p.xs_r) + ((EPI == EPI_SWIGLU && sh) ? (size_t)mt * BM : row0);
       }
+      // training forward: U | V rows of this tile (row 0 of the tile)
+      uint16_t* uv0 = (EPI == EPI_SWIGLU && (sh ? p.uv_s : p.uv_r))
+                          ? (sh ? p.uv_s : p.uv_r) + row0 * (size_t)(2 * ncols) : nullptr;
       if (EPI != EPI_ROUTER && w.n16) {
         epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb,
-                                 xs, wsA, wsB);
+                                 xs, wsA, wsB, uv0);
       } else if (EPI == EPI_ROUTER) {
         // fp32 partial logits of split (nt % ks) for experts of column tile nt / ks
         const int ks = nt % p.r_ks, ct = nt / p.r_ks;
@@ -515,6 +530,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
               const bool in = col0 + v < ncols;
               gv[v] *= rs * (in ? __ldg(wsA + col0 + v) : 0.0f);
               uv[v] *= rs * (in ? __ldg(wsB + col0 + v) : 0.0f);
+            }
+          }
+          if (valid && uv0) {
+            uint16_t* uvr = uv0 + (size_t)r * 2 * ncols;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col0 + 8 * v < ncols) {
+                *reinterpret_cast<uint4*>(uvr + col0 + 8 * v) =
+                    make_uint4(pack_bf16(gv[8 * v], gv[8 * v + 1]), pack_bf16(gv[8 * v + 2], gv[8 * v + 3]),
+                               pack_bf16(gv[8 * v + 4], gv[8 * v + 5]), pack_bf16(gv[8 * v + 6], gv[8 * v + 7]));
+                *reinterpret_cast<uint4*>(uvr + ncols + col0 + 8 * v) =
+                    make_uint4(pack_bf16(uv[8 * v], uv[8 * v + 1]), pack_bf16(uv[8 * v + 2], uv[8 * v + 3]),
+                               pack_bf16(uv[8 * v + 4], uv[8 * v + 5]), pack_bf16(uv[8 * v + 6], uv[8 * v + 7]));
+              }
             }
           }
           if (valid) {
@@ -567,7 +596,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         tc_fence_after();
         epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
                                  tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
-                                 xs ? xs + BM : nullptr, wsA, wsB);
+                                 xs ? xs + BM : nullptr, wsA, wsB, uv0 ? uv0 + (size_t)BM * 2 * ncols : nullptr);
         tc_fence_before();
         mbar_arrive(&acc_empty[1]);
       }
@@ -751,6 +780,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
       p.s1_s = has_s ? blob_scales(a.wu_s, wr_s, a.d) : p.s1_r;
     }
     p.prefix = a.pre_gu;
+    p.uv_r = (uint16_t*)a.uv_r; p.uv_s = (uint16_t*)(has_s ? a.uv_s : a.uv_r);
     p.k_r = p.k_s = a.d;
     p.wrows_r = a.f_r; p.wrows_s = a.f_s;
     p.ncols_r = a.f_r; p.ncols_s = a.f_s;

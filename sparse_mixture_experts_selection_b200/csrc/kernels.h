@@ -26,6 +26,8 @@ struct FfnArgs {
   const float *xs_r, *xs_s;
   void *actq_r, *actq_s;
   float *as_r, *as_s;
+  // training forward: U | V of every row ([rows, 2f] bf16) for the backward
+  void *uv_r, *uv_s;
 };
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
@@ -80,6 +82,40 @@ constexpr int kRouterMaxKbPerSplit = 24;
 void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per);
 cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpart, int T, int d,
                              int E, int* err, int* ks_out, cudaStream_t st);
+
+// Backward of the grouped SwiGLU experts (tcgen05, bf16): which 0 = dU|dV from
+// dO and W_d; 1 = dX from dU|dV and W_g, W_u; 2, 3, 4 = dW_d, dW_g, dW_u.
+// Routed rows are the permuted rows (grp_rows / grp_row0 of the routed
+// groups); shared groups cover all T tokens (rows j*T.. of their buffers).
+struct BwdArgs {
+  int T, d, f_r, f_s, E_r, E_s, max_rows_r;
+  const void *dO_r, *dy;                 // g*dy per permuted row [R, d]; dy [T, d]
+  const void *wg_r, *wu_r, *wd_r, *wg_s, *wu_s, *wd_s;
+  const void *uv_r, *uv_s;               // saved U | V [rows, 2f]
+  void *duv_r, *duv_s;                   // dU | dV [rows, 2f]
+  void *dx_r, *dx_s;                     // dX [rows, d]
+  const void *x_r, *h;                   // permuted rows x [R, d]; h [T, d]
+  const void *act_r, *act_s;             // A = SiLU(U) V [rows, f]
+  void *dwg_r, *dwu_r, *dwd_r, *dwg_s, *dwu_s, *dwd_s;
+  const int *grp_rows, *grp_row0, *pre_da, *pre_dx;
+  int* err;
+};
+cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st);
+
+// Backward of routing and combine (bf16 activations): per permuted row dO and
+// dL/dg; per token dz, dh; per expert de.
+struct BwdRouteArgs {
+  int T, d, E, K, E_s, score_fn, add_residual, max_rows;
+  const uint16_t *dy, *slot, *dx_r, *dx_s, *h;
+  const int32_t *perm_tok, *row_of, *idx;
+  const int* n_rows_ptr;
+  const float *row_gate, *s, *e;
+  uint16_t *dO, *dh;
+  float *dg_row, *dz, *de;
+  int* err;
+};
+void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st);        // dO, dL/dg
+void launch_bwd_gate_dh_de(const BwdRouteArgs& a, cudaStream_t st);   // dz, dh, de
 
 int tc_bm();
 int tc_merge_rows();   // tails of <= this many rows share the unit of the tile before

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     for s in syms:
         assert hasattr(L, s), s
     assert set(syms) == set(moe.SIGNATURES), set(syms) ^ set(moe.SIGNATURES)
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
     assert moe.lib().moe_status_string(3) == b"MOE_ERR_WORKSPACE"
 
 
