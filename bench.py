@@ -221,6 +221,159 @@ def oracle_sample_time(w, tokens: np.ndarray, step: int = 0):
     return time.perf_counter() - t0
 
 
+def oracle_train_sample_time(w, tokens: np.ndarray):
+    """Time the oracle's layer forward + backward on a sample of tokens (the
+    layer restricted to them, full-size experts; weights generated before the
+    clock starts)."""
+    from moe_inputs import native
+    from oracle import moe_oracle as mo
+    h = np.stack([mi.gen_h(w, 0, slice(int(t), int(t) + 1))[0] for t in tokens])
+    e, b = mi.gen_centroids(w), mi.gen_bias(w)
+    cfg = mo.LayerConfig(T=len(tokens), d_model=w.d_model, E_r=w.E_r, E_s=w.E_s, K=w.K,
+                         score_fn=w.score_fn, n_groups=w.n_groups, topk_groups=w.topk_groups,
+                         group_topn=w.group_topn, capacity_factor=w.capacity_factor,
+                         add_residual=w.add_residual)
+    s = mo.affinity(h, e, w.score_fn)
+    idx = mo.select_experts(s, b, w.K, w.n_groups, w.topk_groups, w.group_topn)
+    need = [(which, int(ex)) for ex in np.unique(idx) for which in ("gate", "up", "down")]
+    need += [(which, j) for j in range(w.E_s) for which in ("sgate", "sup", "sdown")]
+    W = {key: native.weight_host(w, *key) for key in need}
+    src = lambda which, ex: W[(which, int(ex))]
+    dy = np.random.default_rng(5).normal(size=h.shape)
+    t0 = time.perf_counter()
+    out = mo.layer_forward(cfg, h, e, b, src)
+    _, gates, disp = mo.route(cfg, out["s"], b if w.score_fn == 0 else np.zeros(w.E_r, np.float32))
+    mo.layer_backward(cfg, h, e, out["s"], out["idx"], gates, disp, src, dy)
+    return time.perf_counter() - t0
+
+
+def train_work(w, kept: np.ndarray):
+    """(flops, bytes) of one backward: dA, dX and the weight gradients of every
+    kept row and shared row, and the router terms; reads of every touched
+    expert's weights, a write of every expert's weight gradient (zero for
+    untouched ones), dy in, dh and de out."""
+    n_rows = int(kept.sum())
+    touched = int((kept > 0).sum())
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    flops = 12 * d * (f * n_rows + fs * w.E_s * w.T) + 4 * w.T * w.E_r * d
+    nbytes = (touched * 3 * d * f * 2 + w.E_r * 3 * d * f * 2 + 2 * w.E_s * 3 * d * fs * 2
+              + 3 * w.T * d * 2 + w.E_r * d * 4)
+    return flops, nbytes
+
+
+def run_train(args, w, rank, world, local_rank):
+    """Training step: moe_layer_forward (train = 1) + moe_layer_backward."""
+    import torch
+    import torch.distributed as dist
+    import sparse_mixture_experts_selection_b200 as moe
+    from moe_inputs import native
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    W, G = {}, {}
+    for k in ("gate", "up", "down", "sgate", "sup", "sdown"):
+        tid, n, rows, cols, sigma = mi.weight_spec(w, k)
+        if n == 0:
+            W[k] = G[k] = None
+            continue
+        W[k] = torch.empty((n, rows, cols), dtype=torch.bfloat16, device=dev)
+        native.fill_device(W[k].data_ptr(), W[k].numel(), True, w.seed, tid, 0, sigma, stream=stream.cuda_stream)
+        G[k] = torch.empty_like(W[k])
+    e = torch.from_numpy(mi.gen_centroids(w)).to(dev)
+    b = torch.from_numpy(mi.gen_bias(w)).to(dev)
+    n_steps = args.warmup + args.steps
+    H = []
+    for i in range(n_steps):
+        t = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device=dev)
+        native.fill_device(t.data_ptr(), t.numel(), True, w.seed, h_stream_id(rank, i), 0, 1.0,
+                           stream=stream.cuda_stream)
+        H.append(t)
+    dy = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device=dev)
+    native.fill_device(dy.data_ptr(), dy.numel(), True, w.seed, 77, 0, 1.0, stream=stream.cuda_stream)
+    cfg = moe.config_for(w, train=1)
+    ws = moe.alloc_workspace(moe.moe_workspace_size(cfg), dev)
+    y = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device=dev)
+    s_out = torch.empty((w.T, w.E_r), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.T, w.K), dtype=torch.int32, device=dev)
+    kept = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
+    dh = torch.empty_like(y)
+    de = torch.empty((w.E_r, w.d_model), dtype=torch.float32, device=dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_steps)]
+
+    def step(i):
+        ev[i][0].record()
+        moe.moe_layer_forward(cfg, H[i], e, b, W["gate"], W["up"], W["down"], W["sgate"], W["sup"],
+                              W["sdown"], y, ws, idx_out=idx, kept_out=kept[i], s_out=s_out,
+                              update_bias=w.gamma > 0, gamma=w.gamma)
+        ev[i][1].record()
+        moe.moe_layer_backward(cfg, H[i], e, s_out, idx, W["gate"], W["up"], W["down"], W["sgate"],
+                               W["sup"], W["sdown"], dy, dh, de, G["gate"], G["up"], G["down"],
+                               G["sgate"], G["sup"], G["sdown"], ws)
+        ev[i][2].record()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    t0.record()
+    for j in range(args.steps):
+        step(args.warmup + j)
+    t1.record()
+    torch.cuda.synchronize()
+    clocks.mark(wall0, time.time())
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    err = moe.moe_get_device_error(ws)
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed region")
+    fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, n_steps)]
+    bwd = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.warmup, n_steps)]
+    kept_h = kept.cpu().numpy()[args.warmup:]
+    clk = clocks.summary()
+    clocks.stop()
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    hbm, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops_sustained"])
+    tw = [train_work(w, k) for k in kept_h]
+    b_flops, b_bytes = float(np.mean([x[0] for x in tw])), float(np.mean([x[1] for x in tw]))
+    bwd_s = float(np.mean(bwd)) / 1000
+    t_roof_b = max(b_flops / (bf16_peak * 1e12), b_bytes / (hbm * 1e9))
+    ms_per_step = elapsed_ms / args.steps
+    line = {
+        "metric": "MoE-layer training step (forward + backward) tokens/s", "value": job_throughput(world, w.T, args.steps, elapsed_ms),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w), step="moe_layer_forward (train) + moe_layer_backward",
+                       parallelism=f"replicas x{world}"),
+        "forward_ms": float(np.mean(fwd)), "backward_ms": float(np.mean(bwd)),
+        "backward_roofline": {"t_roof_ms": 1000 * t_roof_b, "frac": 1000 * t_roof_b / float(np.mean(bwd)),
+                              "flops": b_flops, "bytes": b_bytes,
+                              "bound": "hbm" if b_bytes / (hbm * 1e9) >= b_flops / (bf16_peak * 1e12) else "tensor",
+                              "achieved_gbs": b_bytes / bwd_s / 1e9, "achieved_tflops": b_flops / bwd_s / 1e12,
+                              "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained"},
+        "clocks": clk,
+        # forward 11 + backward: groups, rows, 5 GEMMs, gates, dh, de
+        "gpu_launches": 21 * args.steps,
+    }
+    if not args.no_cpu_baseline:
+        n_tok = 2
+        rng = np.random.default_rng(12345)
+        tokens = np.sort(rng.choice(w.T, size=n_tok, replace=False))
+        dt = oracle_train_sample_time(w, tokens)
+        line["cpu_baseline"] = {"value": n_tok / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n_tok} seeded tokens: layer forward + backward restricted to "
+                                          f"them, full-size experts, float64 numpy"}
+    print(json.dumps(line), flush=True)
+
+
 def cpu_baseline(w, n_tokens: int):
     rng = np.random.default_rng(12345)
     tokens = np.sort(rng.choice(w.T, size=n_tokens, replace=False))
@@ -522,6 +675,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--train", action="store_true",
+                    help="time the training step (forward with train = 1 + moe_layer_backward)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling only: tokens per step (with --experts)")
     ap.add_argument("--experts", type=int, default=0,
@@ -549,7 +704,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if args.train:
+            run_train(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

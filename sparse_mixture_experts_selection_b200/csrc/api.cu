@@ -48,6 +48,8 @@ struct Layout {
   size_t xs, hq, hs, actq_r, actq_s, as_r, as_s;
   // training: U | V kept by the forward; the backward's dO, dL/dg, dz, dU | dV, dX
   size_t uv_r, uv_s, dO, dg_row, dz, duv_r, duv_s, dx_r, dx_s;
+  // every selected (token, expert) pair by expert (dropped ones included)
+  size_t sel_tok, sel_row_of, sel_off, sel_base, sel_counts, sel_kept;
   size_t total;
   int n_chunks;
   int64_t cap, R;
@@ -109,6 +111,12 @@ Layout make_layout(const moe_config& c) {
   L.duv_s = take(tr ? rs * 2 * fs * 2 : 0);
   L.dx_r = take(tr ? (size_t)L.R * c.d_model * 2 : 0);
   L.dx_s = take(tr ? rs * c.d_model * 2 : 0);
+  L.sel_tok = take(tr ? (size_t)c.T * c.K * 4 : 0);
+  L.sel_row_of = take(tr ? (size_t)c.T * c.K * 4 : 0);
+  L.sel_off = take(tr ? (size_t)(c.E_r + 1) * 4 : 0);
+  L.sel_base = take(tr ? (size_t)L.n_chunks * c.E_r * 4 : 0);
+  L.sel_counts = take(tr ? (size_t)c.E_r * 4 : 0);
+  L.sel_kept = take(tr ? (size_t)c.E_r * 4 : 0);
   L.total = o;
   return L;
 }
@@ -549,6 +557,17 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float*
   ra.dO = at<uint16_t>(ws, L.dO); ra.dh = static_cast<uint16_t*>(dh);
   ra.dg_row = at<float>(ws, L.dg_row); ra.dz = at<float>(ws, L.dz); ra.de = de;
   ra.err = err;
+  if (c.score_fn == MOE_SCORE_SIGMOID) {
+    // the forward's per-chunk histogram, scanned without a capacity and
+    // scattered stably: every selected pair by expert, tokens ascending
+    const int all = c.T * c.K;
+    moe::launch_scan(at<int>(ws, L.hist), L.n_chunks, c.E_r, all, at<int>(ws, L.sel_counts),
+                     at<int>(ws, L.sel_kept), at<int>(ws, L.sel_off), at<int>(ws, L.sel_base), st);
+    moe::launch_scatter(idx, nullptr, at<int>(ws, L.sel_off), at<int>(ws, L.sel_base), all, c.T, c.K, c.E_r,
+                        at<int32_t>(ws, L.sel_tok), at<int32_t>(ws, L.sel_row_of), nullptr, err, st);
+    ra.sel_tok = at<int32_t>(ws, L.sel_tok);
+    ra.sel_off = at<int>(ws, L.sel_off);
+  }
   moe::launch_bwd_route(ra, st);                      // dO = g dy, dL/dg per kept row
   moe::BwdArgs ba{};
   ba.T = c.T; ba.d = c.d_model; ba.f_r = c.d_ffn; ba.f_s = fs; ba.E_r = c.E_r; ba.E_s = c.E_s;

@@ -118,8 +118,9 @@ bwd_gate_kernel(const float* __restrict__ s, const int32_t* __restrict__ idx,
 __global__ void __launch_bounds__(256)
 bwd_dh_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ dx_r,
               const uint16_t* __restrict__ dx_s, const int32_t* __restrict__ row_of,
-              const float* __restrict__ dz, const float* __restrict__ e, int T, int d, int K, int E,
-              int E_s, int add_residual, int n_rows, uint16_t* __restrict__ dh) {
+              const float* __restrict__ dz, const float* __restrict__ e, const int32_t* __restrict__ idx,
+              int T, int d, int K, int E, int E_s, int add_residual, int n_rows, int sparse,
+              uint16_t* __restrict__ dh) {
   const int t = blockIdx.x;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     float acc[8], v[8];
@@ -138,8 +139,12 @@ bwd_dh_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ dx_r
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += v[i];
     }
+    // router term: sigmoid routing has dz != 0 only on the K selected experts
+    // (ascending, as idx stores them); softmax touches every expert
     const float* zr = dz + (size_t)t * E;
-    for (int j = 0; j < E; ++j) {
+    const int nj = sparse ? K : E;
+    for (int q = 0; q < nj; ++q) {
+      const int j = sparse ? idx[(size_t)t * K + q] : q;
       const float z = zr[j];
       if (z == 0.0f) continue;
       const float4 e0 = *reinterpret_cast<const float4*>(e + (size_t)j * d + c);
@@ -169,6 +174,26 @@ bwd_de_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ h, int 
   if (c < d) de[(size_t)j * d + c] = acc;
 }
 
+// de for sigmoid routing: dz is non-zero only on the selected pairs; the
+// pairs of expert j (every selected (t, j), dropped ones included) are rows
+// sel_off[j] .. sel_off[j+1] of sel_tok, in ascending token order.
+__global__ void __launch_bounds__(256)
+bwd_de_sparse_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ h,
+                     const int32_t* __restrict__ sel_tok, const int* __restrict__ sel_off, int T, int d,
+                     int E, float* __restrict__ de) {
+  const int j = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  float acc = 0.0f;
+  const int r0 = sel_off[j], r1 = sel_off[j + 1];
+  for (int r = r0; r < r1; ++r) {
+    const int t = sel_tok[r];
+    if (t < 0 || t >= T) continue;
+    const float z = __ldg(dz + (size_t)t * E + j);
+    if (c < d) acc = fmaf(z, __uint_as_float((uint32_t)h[(size_t)t * d + c] << 16), acc);
+  }
+  if (c < d) de[(size_t)j * d + c] = acc;
+}
+
 }  // namespace
 
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st) {
@@ -179,9 +204,14 @@ void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st) {
 
 void launch_bwd_gate_dh_de(const BwdRouteArgs& a, cudaStream_t st) {
   bwd_gate_kernel<<<(a.T + 7) / 8, 256, 0, st>>>(a.s, a.idx, a.row_of, a.dg_row, a.score_fn, a.T, a.E, a.K, a.dz);
-  bwd_dh_kernel<<<a.T, 256, 0, st>>>(a.dy, a.dx_r, a.dx_s, a.row_of, a.dz, a.e, a.T, a.d, a.K, a.E, a.E_s,
-                                     a.add_residual, a.max_rows, a.dh);
-  bwd_de_kernel<<<dim3(a.E, (a.d + 255) / 256), 256, 0, st>>>(a.dz, a.h, a.T, a.d, a.E, a.de);
+  const int sparse = a.score_fn == 0;
+  bwd_dh_kernel<<<a.T, 256, 0, st>>>(a.dy, a.dx_r, a.dx_s, a.row_of, a.dz, a.e, a.idx, a.T, a.d, a.K, a.E,
+                                     a.E_s, a.add_residual, a.max_rows, sparse, a.dh);
+  if (sparse)
+    bwd_de_sparse_kernel<<<dim3(a.E, (a.d + 255) / 256), 256, 0, st>>>(a.dz, a.h, a.sel_tok, a.sel_off, a.T,
+                                                                       a.d, a.E, a.de);
+  else
+    bwd_de_kernel<<<dim3(a.E, (a.d + 255) / 256), 256, 0, st>>>(a.dz, a.h, a.T, a.d, a.E, a.de);
 }
 
 }  // namespace moe

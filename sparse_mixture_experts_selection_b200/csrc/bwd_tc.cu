@@ -41,6 +41,11 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int UNIT_RING = 4;
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512;
+// EPI_DW: 3 stages (an expert has few k-blocks) and a 64 KB staging buffer for
+// the output tile, written back by TMA stores (4 warps x 4 boxes of 64 x 32)
+constexpr int DW_STAGES = 3;
+constexpr int DW_OUT_BYTES = BM * BN * 2;
+constexpr size_t DW_SMEM_BYTES = (size_t)DW_STAGES * STAGE_BYTES + DW_OUT_BYTES + 1024 + 512;
 
 enum { EPI_DA = 0, EPI_DX = 1, EPI_DW = 2 };
 
@@ -64,6 +69,7 @@ struct Params {
   int a_x0_r, a_x0_s;                    // column offset into A's rows (dW_u: the V half, f)
   uint16_t* dw_r;                        // [E, M, N] bf16
   uint16_t* dw_s;
+  CUtensorMap dws_r, dws_s;              // EPI_DW store maps over [E, M, N], box {64, 32, 1}
   int* err;
 };
 
@@ -163,13 +169,23 @@ __device__ __forceinline__ void load_stage(const Params& p, const Unit& w, int i
   }
 }
 
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               :: "l"(tmap), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_constant__ Params p) {
+  constexpr int STAGES = EPI == EPI_DW ? DW_STAGES : bwd::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sOut = smem + STAGES * STAGE_BYTES;                  // EPI_DW staging (1024-aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + (EPI == EPI_DW ? DW_OUT_BYTES : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -306,33 +322,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       if (EPI == EPI_DW) {
-        // weight-gradient tile: row mt*128 + r of the expert's [M, N] matrix
-        const int M = w.sh ? p.M_s : p.M_r, N = w.sh ? p.N_s : p.N_r;
-        const int e = w.sh ? w.g - p.E_r : w.g;
-        const int m = w.mt * BM + r;
-        uint16_t* dst = (w.sh ? p.dw_s : p.dw_r) + ((size_t)e * M + m) * N;
+        // weight-gradient tile, rows sub*32.. of the tile: staged in this warp's
+        // 16 KB of sOut as four 64 x 32 boxes in the 128-byte swizzle layout the
+        // store map expects (16-byte chunk j of line r at chunk j ^ (r & 7)),
+        // then written by TMA stores that clip at the expert's M and N
+        uint8_t* stg = sOut + sub * (DW_OUT_BYTES / 4);
+        if (lane == 0) bulk_wait_read();               // the previous tile's stores have read stg
+        __syncwarp();
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float dv[32];
           tmem_ld32(tb + c, dv);
-          const int col0 = w.nt * BN + c;
-          if (m < M) {
+          uint8_t* line = stg + (c / 64) * 4096 + lane * 128;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col0 + 8 * v < N) {
-                uint4 pk;
-                if (w.nk == 0) pk = make_uint4(0, 0, 0, 0);     // an expert without rows
-                else {
-                  pk.x = pack_bf16(dv[8 * v + 0], dv[8 * v + 1]);
-                  pk.y = pack_bf16(dv[8 * v + 2], dv[8 * v + 3]);
-                  pk.z = pack_bf16(dv[8 * v + 4], dv[8 * v + 5]);
-                  pk.w = pack_bf16(dv[8 * v + 6], dv[8 * v + 7]);
-                }
-                *reinterpret_cast<uint4*>(dst + col0 + 8 * v) = pk;
-              }
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            if (w.nk == 0) pk = make_uint4(0, 0, 0, 0);        // an expert without rows
+            else {
+              pk.x = pack_bf16(dv[8 * v + 0], dv[8 * v + 1]);
+              pk.y = pack_bf16(dv[8 * v + 2], dv[8 * v + 3]);
+              pk.z = pack_bf16(dv[8 * v + 4], dv[8 * v + 5]);
+              pk.w = pack_bf16(dv[8 * v + 6], dv[8 * v + 7]);
             }
+            const int chunk = ((c % 64) / 8 + v) ^ (lane & 7);
+            *reinterpret_cast<uint4*>(line + chunk * 16) = pk;
           }
         }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[acc]);                  // TMEM is free; the stores go on
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int e = w.sh ? w.g - p.E_r : w.g;
+          const CUtensorMap* dm = w.sh ? &p.dws_s : &p.dws_r;
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q)
+            tma_store_3d(dm, stg + q * 4096, w.nt * BN + q * 64, w.mt * BM + sub * 32, e);
+          bulk_commit();
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
       } else {
         const int m = w.mt * BM + r;
         const bool valid = m < w.rows;
@@ -391,6 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     }
   }
 
+  if (EPI == EPI_DW && warp >= 2 && lane == 0) bulk_wait_all();   // every TMA store has landed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -427,6 +458,19 @@ static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 tensor [n, rows, cols] for TMA stores; box = 64 columns x 32 rows x 1
+static bool make_store_map(CUtensorMap* m, const void* base, uint64_t n, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || !base) return false;
+  cuuint64_t dims[3] = {cols, rows, n < 1 ? 1 : n};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -439,12 +483,13 @@ static cudaError_t launch(const Params& p, int units, cudaStream_t st) {
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
+  const size_t smem = EPI == EPI_DW ? DW_SMEM_BYTES : SMEM_BYTES;
   if (dev < 64 && !attr_done[dev]) {
-    cudaFuncSetAttribute(bwd_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(bwd_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attr_done[dev] = true;
   }
   const int grid = std::max(1, std::min(units, num_sms()));
-  bwd_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  bwd_gemm_kernel<EPI><<<grid, NUM_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -520,6 +565,9 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st) {
     p.dw_r = (uint16_t*)(up ? a.dwu_r : a.dwg_r); p.dw_s = (uint16_t*)(up ? a.dwu_s : a.dwg_s);
   }
   p.b1_r = p.b0_r; p.b1_s = p.b0_s;
+  ok &= make_store_map(&p.dws_r, p.dw_r, (uint64_t)a.E_r, p.M_r, p.N_r);
+  ok &= make_store_map(&p.dws_s, has_s ? (const void*)p.dw_s : (const void*)p.dw_r, (uint64_t)(has_s ? a.E_s : a.E_r),
+                       has_s ? p.M_s : p.M_r, has_s ? p.N_s : p.N_r);
   p.mt_r = (p.M_r + BM - 1) / BM; p.nt_r = (p.N_r + BN - 1) / BN;
   p.mt_s = (p.M_s + BM - 1) / BM; p.nt_s = (p.N_s + BN - 1) / BN;
   if (!ok) return cudaErrorInvalidValue;

@@ -112,6 +112,8 @@ struct BwdRouteArgs {
   const float *row_gate, *s, *e;
   uint16_t *dO, *dh;
   float *dg_row, *dz, *de;
+  const int32_t* sel_tok;    // sigmoid: every selected (t, j) by expert, tokens ascending
+  const int* sel_off;        // [E + 1] its offsets
   int* err;
 };
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st);        // dO, dL/dg
