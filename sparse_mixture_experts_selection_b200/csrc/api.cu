@@ -585,6 +585,10 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float*
   ba.grp_rows = at<int>(ws, L.grp_rows); ba.grp_row0 = at<int>(ws, L.grp_row0);
   ba.pre_da = at<int>(ws, L.pre_gu); ba.pre_dx = at<int>(ws, L.pre_dn);
   ba.err = err;
+  // operand B of the weight gradients (x, A) is read up to 63 rows past the
+  // last routed row: keep those rows finite (zero)
+  moe::launch_zero_tail_rows(at<void>(ws, L.x_perm), offsets + c.E_r, R, c.d_model, st);
+  moe::launch_zero_tail_rows(at<void>(ws, L.act_r), offsets + c.E_r, R, c.d_ffn, st);
   for (int which = 0; which < 5; ++which) {
     cudaError_t er = moe::launch_bwd_tc(ba, which, st);
     if (er != cudaSuccess) return fail(MOE_ERR_CUDA, "backward GEMM %d: %s", which, cudaGetErrorString(er));

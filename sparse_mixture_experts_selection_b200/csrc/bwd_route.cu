@@ -194,7 +194,24 @@ bwd_de_sparse_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ 
   if (c < d) de[(size_t)j * d + c] = acc;
 }
 
+// Zero rows n .. n+63 (n = *n_rows_ptr, capped at max_rows) of a bf16 [max_rows, cols]
+// buffer: the weight-gradient GEMMs read up to 63 lines past an expert's last
+// row as operand B, which must be finite there.
+__global__ void zero_tail_rows_kernel(uint16_t* __restrict__ buf, const int* __restrict__ n_rows_ptr,
+                                      int max_rows, int cols) {
+  const int n = min(*n_rows_ptr, max_rows);
+  const int rows = min(64, max_rows - n);
+  const size_t total = (size_t)rows * cols / 8;
+  uint4* p = reinterpret_cast<uint4*>(buf + (size_t)n * cols);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x)
+    p[i] = make_uint4(0, 0, 0, 0);
+}
+
 }  // namespace
+
+void launch_zero_tail_rows(void* buf, const int* n_rows_ptr, int max_rows, int cols, cudaStream_t st) {
+  zero_tail_rows_kernel<<<64, 256, 0, st>>>(static_cast<uint16_t*>(buf), n_rows_ptr, max_rows, cols);
+}
 
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st) {
   const int warps = a.max_rows < 148 * 64 ? (a.max_rows > 0 ? a.max_rows : 1) : 148 * 64;

@@ -42,7 +42,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int UNIT_RING = 4;
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512;
 // EPI_DW: 3 stages (an expert has few k-blocks) and a 64 KB staging buffer for
-// the output tile, written back by TMA stores (4 warps x 4 boxes of 64 x 32)
+// the output tile, written back by TMA stores (4 boxes of 64 columns x 128 rows)
 constexpr int DW_STAGES = 3;
 constexpr int DW_OUT_BYTES = BM * BN * 2;
 constexpr size_t DW_SMEM_BYTES = (size_t)DW_STAGES * STAGE_BYTES + DW_OUT_BYTES + 1024 + 512;
@@ -69,7 +69,7 @@ struct Params {
   int a_x0_r, a_x0_s;                    // column offset into A's rows (dW_u: the V half, f)
   uint16_t* dw_r;                        // [E, M, N] bf16
   uint16_t* dw_s;
-  CUtensorMap dws_r, dws_s;              // EPI_DW store maps over [E, M, N], box {64, 32, 1}
+  CUtensorMap dws_r, dws_s;              // EPI_DW store maps over [E, M, N], box {64, 128, 1}
   int* err;
 };
 
@@ -177,6 +177,7 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_constant__ Params p) {
   constexpr int STAGES = EPI == EPI_DW ? DW_STAGES : bwd::STAGES;
@@ -190,7 +191,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* unit_full = drain + 1;
+  uint64_t* stg_full = drain + 1;        // EPI_DW: the staged tile is complete (128 arrivals)
+  uint64_t* stg_free = stg_full + 1;     // EPI_DW: the previous tile's stores have read sOut
+  uint64_t* unit_full = stg_free + 1;
   uint64_t* unit_empty = unit_full + UNIT_RING;
   volatile int* unit_ring = reinterpret_cast<volatile int*>(unit_empty + UNIT_RING);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UNIT_RING);
@@ -202,6 +205,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4 * kWarp); }
     for (int s = 0; s < UNIT_RING; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1 + 4 * kWarp); }
     mbar_init(drain, 1);
+    mbar_init(stg_full, 4 * kWarp);
+    mbar_init(stg_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -268,13 +273,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
         if (EPI == EPI_DW) {
           const int valid = w.rows - kb * BK;           // K-lines that belong to the group
           if (valid < BK) {
-            // zero lines valid..63 of every 64-element MN block of A (2) and B (4)
-            const int lines = BK - valid;
-            for (int q = lane; q < lines * 6 * 8; q += kWarp) {
-              const int blk = q / (lines * 8), rem = q % (lines * 8);
-              const int line = valid + rem / 8, chunk = rem % 8;
-              uint8_t* base = blk < 2 ? a_st + blk * MN_BOX_BYTES : b_st + (blk - 2) * MN_BOX_BYTES;
-              *reinterpret_cast<uint4*>(base + line * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+            // zero lines valid..63 of A's two 64-element MN blocks: with those
+            // lines zero, B's lines past the group (the next group's rows, the
+            // zeroed rows after the last routed row, or TMA's zero fill) add nothing
+            for (int line = valid + (lane >> 3); line < BK; line += kWarp / 8) {
+              *reinterpret_cast<uint4*>(a_st + line * 128 + (lane & 7) * 16) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4*>(a_st + MN_BOX_BYTES + line * 128 + (lane & 7) * 16) = make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
           }
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
     int acc = 0, slot = 0;
-    uint32_t acc_phase = 0, uphase = 0;
+    uint32_t acc_phase = 0, uphase = 0, stg_phase = 0;
     for (;;) {
       if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
       const int u = unit_ring[slot];
@@ -322,18 +326,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       if (EPI == EPI_DW) {
-        // weight-gradient tile, rows sub*32.. of the tile: staged in this warp's
-        // 16 KB of sOut as four 64 x 32 boxes in the 128-byte swizzle layout the
-        // store map expects (16-byte chunk j of line r at chunk j ^ (r & 7)),
-        // then written by TMA stores that clip at the expert's M and N
-        uint8_t* stg = sOut + sub * (DW_OUT_BYTES / 4);
-        if (lane == 0) bulk_wait_read();               // the previous tile's stores have read stg
-        __syncwarp();
+        // weight-gradient tile staged in sOut as four 128-row x 64-column boxes
+        // in the 128-byte swizzle layout the store map expects (16-byte chunk j
+        // of line r at chunk j ^ (r & 7)); this warp writes lines sub*32.. of
+        // each box, then one thread writes the four boxes by TMA stores that
+        // clip at the expert's M and N
+        const bool leader = warp == 2 && lane == 0;
+        if (leader) {
+          bulk_wait_read();                            // the previous tile's stores have read sOut
+          mbar_arrive(stg_free);
+        }
+        if (!mbar_wait(stg_free, stg_phase, abort_flag, p.err)) break;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float dv[32];
           tmem_ld32(tb + c, dv);
-          uint8_t* line = stg + (c / 64) * 4096 + lane * 128;
+          uint8_t* line = sOut + (c / 64) * (DW_OUT_BYTES / 4) + r * 128;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pk;
@@ -344,22 +352,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
               pk.z = pack_bf16(dv[8 * v + 4], dv[8 * v + 5]);
               pk.w = pack_bf16(dv[8 * v + 6], dv[8 * v + 7]);
             }
-            const int chunk = ((c % 64) / 8 + v) ^ (lane & 7);
+            const int chunk = ((c % 64) / 8 + v) ^ (r & 7);
             *reinterpret_cast<uint4*>(line + chunk * 16) = pk;
           }
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);                  // TMEM is free; the stores go on
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
+        mbar_arrive(stg_full);
+        if (leader) {
+          if (!mbar_wait(stg_full, stg_phase, abort_flag, p.err)) break;
           const int e = w.sh ? w.g - p.E_r : w.g;
           const CUtensorMap* dm = w.sh ? &p.dws_s : &p.dws_r;
 #pragma unroll
           for (int q = 0; q < BN / 64; ++q)
-            tma_store_3d(dm, stg + q * 4096, w.nt * BN + q * 64, w.mt * BM + sub * 32, e);
+            tma_store_3d(dm, sOut + q * (DW_OUT_BYTES / 4), w.nt * BN + q * 64, w.mt * BM, e);
           bulk_commit();
         }
+        stg_phase ^= 1u;
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
         continue;
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     }
   }
 
-  if (EPI == EPI_DW && warp >= 2 && lane == 0) bulk_wait_all();   // every TMA store has landed
+  if (EPI == EPI_DW && warp == 2 && lane == 0) bulk_wait_all();   // every TMA store has landed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -458,13 +468,13 @@ static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 tensor [n, rows, cols] for TMA stores; box = 64 columns x 32 rows x 1
+// bf16 tensor [n, rows, cols] for TMA stores; box = 64 columns x 128 rows x 1
 static bool make_store_map(CUtensorMap* m, const void* base, uint64_t n, uint64_t rows, uint64_t cols) {
   EncodeTiledFn enc = get_encode();
   if (!enc || !base) return false;
   cuuint64_t dims[3] = {cols, rows, n < 1 ? 1 : n};
   cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
-  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,

@@ -117,6 +117,7 @@ struct BwdRouteArgs {
   int* err;
 };
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st);        // dO, dL/dg
+void launch_zero_tail_rows(void* buf, const int* n_rows_ptr, int max_rows, int cols, cudaStream_t st);
 void launch_bwd_gate_dh_de(const BwdRouteArgs& a, cudaStream_t st);   // dz, dh, de
 
 int tc_bm();
