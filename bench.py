@@ -360,8 +360,9 @@ def run_train(args, w, rank, world, local_rank):
                               "achieved_gbs": b_bytes / bwd_s / 1e9, "achieved_tflops": b_flops / bwd_s / 1e12,
                               "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained"},
         "clocks": clk,
-        # forward 11 + backward: groups, rows, 5 GEMMs, gates, dh, de
-        "gpu_launches": 21 * args.steps,
+        # forward 11 + backward: groups, (sigmoid: scan + scatter of every selected
+        # pair), 2 tail zeroings, rows, 5 GEMMs, gates, dh, de
+        "gpu_launches": (11 + 12 + (2 if w.score_fn == 0 else 0)) * args.steps,
     }
     if not args.no_cpu_baseline:
         n_tok = 2
