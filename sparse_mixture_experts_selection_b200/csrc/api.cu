@@ -541,8 +541,9 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float*
   const int* offsets = at<int>(ws, L.offsets);
   const int fs = c.E_s ? c.d_ffn_shared : c.d_ffn;
   const int R = (int)L.R;
-  // group tables of the backward GEMMs: plain 128-row tiles, 256-column tiles of f (dA) and d (dX)
-  moe::launch_groups(offsets, c.E_r, c.E_s, c.T, 128, 0, (c.d_ffn + 255) / 256, (fs + 255) / 256,
+  // group tables of the backward GEMMs: 128-row tiles (a last tile of <= 64 rows merged into the
+  // one before), 256-column tiles of f (dA) and d (dX)
+  moe::launch_groups(offsets, c.E_r, c.E_s, c.T, 128, moe::bwd_merge_rows(), (c.d_ffn + 255) / 256, (fs + 255) / 256,
                      (c.d_model + 255) / 256, (c.d_model + 255) / 256, at<int>(ws, L.grp_rows),
                      at<int>(ws, L.grp_row0), at<int>(ws, L.pre_gu), at<int>(ws, L.pre_dn), R, err, err + 16, st);
   moe::BwdRouteArgs ra{};

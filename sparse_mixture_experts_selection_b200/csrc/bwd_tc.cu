@@ -40,7 +40,16 @@ constexpr int MN_BOX_BYTES = MN_BOX * BK * 2;   // 8 KB
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int UNIT_RING = 4;
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512;
+// EPI_DA / EPI_DX: a last row tile of <= MERGE_ROWS rows rides in the unit of
+// the full tile before it (transposed: the stage's weight block is the M
+// operand, the tail rows the N operand), so an expert of 129..192 rows stages
+// each weight tile once; the tail rows take T_BYTES per stage (32-row boxes)
+constexpr int MERGE_ROWS = 64;
+constexpr int SUB_ROWS = 32;
+constexpr int SUB_BYTES = SUB_ROWS * BK * 2;
+constexpr int T_BYTES = MERGE_ROWS * BK * 2;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * (STAGE_BYTES + T_BYTES) + 1024 + 512;
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 // EPI_DW: 3 stages (an expert has few k-blocks) and a 64 KB staging buffer for
 // the output tile, written back by TMA stores (4 boxes of 64 columns x 128 rows)
 constexpr int DW_STAGES = 3;
@@ -51,6 +60,7 @@ enum { EPI_DA = 0, EPI_DX = 1, EPI_DW = 2 };
 
 struct Params {
   CUtensorMap a_r, a_s;                  // A operand, routed / shared groups
+  CUtensorMap a32_r, a32_s;              // EPI_DA / EPI_DX: the same rows with a 32-row box (tails)
   CUtensorMap b0_r, b1_r, b0_s, b1_s;    // B operand (EPI_DX: b0 = W_g for k < kb_split, b1 = W_u)
   const int* grp_rows;
   const int* grp_row0;
@@ -75,6 +85,7 @@ struct Params {
 
 struct Unit {
   int g, mt, nt, nk, rows;
+  int tail, t16;                         // EPI_DA / EPI_DX: merged tail rows, MMA N of the tail
   bool sh;
 };
 
@@ -100,6 +111,7 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
     }
     w.rows = __ldg(p.grp_rows + w.g);
     w.nk = (w.rows + BK - 1) / BK;
+    w.tail = w.t16 = 0;
     return w;
   }
   int lo = 0, hi = p.G;
@@ -111,10 +123,14 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
   w.sh = lo >= p.E_r;
   w.rows = __ldg(p.grp_rows + lo);
   const int mtiles = (w.rows + BM - 1) / BM;
+  const int last = w.rows - (mtiles - 1) * BM;
+  const int runits = mtiles - ((mtiles >= 2 && last <= MERGE_ROWS) ? 1 : 0);
   const int local = u - __ldg(p.prefix + lo);
-  w.mt = local % mtiles;
-  w.nt = local / mtiles;
+  w.mt = local % runits;
+  w.nt = local / runits;
   w.nk = ((w.sh ? p.k_s : p.k_r) + BK - 1) / BK;
+  w.tail = (runits < mtiles && w.mt == runits - 1) ? last : 0;
+  w.t16 = (w.tail + 15) & ~15;
   return w;
 }
 
@@ -142,7 +158,7 @@ __device__ __forceinline__ void unpack8(uint4 q, float* v) {
 // Loads of k-block i of unit w into stage buffers sa / sb.
 template <int EPI>
 __device__ __forceinline__ void load_stage(const Params& p, const Unit& w, int i, uint8_t* sa, uint8_t* sb,
-                                           uint64_t* bar) {
+                                           uint8_t* st, uint64_t* bar) {
   const CUtensorMap* am = w.sh ? &p.a_s : &p.a_r;
   const int row0 = __ldg(p.grp_row0 + w.g);
   const int e = w.sh ? w.g - p.E_r : w.g;
@@ -160,6 +176,8 @@ __device__ __forceinline__ void load_stage(const Params& p, const Unit& w, int i
     // A: 128 rows of the group, K-major; B: K-lines of the expert's weight, 256 MN-columns
     const int ay = (EPI == EPI_DA && w.sh && p.a_sh_zero ? 0 : row0) + w.mt * BM;
     tma_load_2d(sa, am, bar, i * BK, ay);
+    for (int q = 0; q * SUB_ROWS < w.t16; ++q)
+      tma_load_2d(st + q * SUB_BYTES, w.sh ? &p.a32_s : &p.a32_r, bar, i * BK, ay + BM + q * SUB_ROWS);
     const int split = w.sh ? p.kb_split_s : p.kb_split_r;
     const bool second = EPI == EPI_DX && i >= split;
     const CUtensorMap* bm = w.sh ? (second ? &p.b1_s : &p.b0_s) : (second ? &p.b1_r : &p.b0_r);
@@ -178,6 +196,45 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 
+// Epilogue of a merged tail (EPI_DA / EPI_DX): TMEM lane r of half h holds
+// output column nt*256 + h*128 + r, accumulator column t the tail row t.
+template <int EPI>
+__device__ __noinline__ void epilogue_tail(const Params& p, const Unit& w, int r, uint32_t tb) {
+  const size_t row0 = (size_t)__ldg(p.grp_row0 + w.g) + (size_t)(w.mt + 1) * BM;
+  const int ncols = w.sh ? p.ncols_s : p.ncols_r;
+  const int ld = w.sh ? p.ld_s : p.ld_r;
+  const int f = w.sh ? p.f_s : p.f_r;
+  uint16_t* out = w.sh ? p.out_s : p.out_r;
+  const uint16_t* uv = EPI == EPI_DA ? (w.sh ? p.uv_s : p.uv_r) : nullptr;
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int col = w.nt * BN + h * (BN / 2) + r;
+#pragma unroll 1
+    for (int c = 0; c < w.t16; c += 32) {
+      float dv[32];
+      tmem_ld32(tb + h * (BN / 2) + c, dv);
+      if (col < ncols) {
+#pragma unroll
+        for (int v = 0; v < 32; ++v) {
+          const int t = c + v;
+          if (t < w.tail) {
+            const size_t row = row0 + t;
+            if (EPI == EPI_DA) {
+              const float uu = __uint_as_float((uint32_t)uv[row * 2 * f + col] << 16);
+              const float vv = __uint_as_float((uint32_t)uv[row * 2 * f + f + col] << 16);
+              const float sg = 1.0f / (1.0f + __expf(-uu));
+              out[row * ld + col] = __bfloat16_as_ushort(__float2bfloat16_rn(dv[v] * vv * sg * (1.0f + uu * (1.0f - sg))));
+              out[row * ld + f + col] = __bfloat16_as_ushort(__float2bfloat16_rn(dv[v] * uu * sg));
+            } else {
+              out[row * ld + col] = __bfloat16_as_ushort(__float2bfloat16_rn(dv[v]));
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_constant__ Params p) {
   constexpr int STAGES = EPI == EPI_DW ? DW_STAGES : bwd::STAGES;
@@ -186,7 +243,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   uint8_t* sOut = smem + STAGES * STAGE_BYTES;                  // EPI_DW staging (1024-aligned)
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + (EPI == EPI_DW ? DW_OUT_BYTES : 0));
+  uint8_t* sT = sOut;                                            // EPI_DA / EPI_DX: merged tails' rows
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES +
+                                               (EPI == EPI_DW ? DW_OUT_BYTES : STAGES * T_BYTES));
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -214,6 +273,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
   if (warp == 1 && lane == 0) {
     prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.b0_r);
     prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
+    if (EPI != EPI_DW) { prefetch_tmap(&p.a32_r); prefetch_tmap(&p.a32_s); }
   }
   tc_fence_before();
   __syncthreads();
@@ -235,10 +295,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
         if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
         if (u < 0) break;
         const Unit w = decode<EPI>(p, u);
+        const uint32_t tx = STAGE_BYTES + ((w.t16 + SUB_ROWS - 1) / SUB_ROWS) * SUB_BYTES;
         for (int i = 0; i < w.nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          load_stage<EPI>(p, w, i, sA + stage * A_BYTES, sB + stage * B_BYTES, &full[stage]);
+          mbar_arrive_expect_tx(&full[stage], tx);
+          load_stage<EPI>(p, w, i, sA + stage * A_BYTES, sB + stage * B_BYTES, sT + stage * T_BYTES,
+                          &full[stage]);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -252,8 +314,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
   } else if (warp == 1) {
     // ---------------- MMA issuer (lane 0; the warp zeroes K tails) ----------------
     constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN) | kIdescBMnMajor | (EPI == EPI_DW ? kIdescAMnMajor : 0u);
-    int stage = 0, acc = 0, slot = 0;
-    uint32_t phase = 0, acc_phase = 0, uphase = 0;
+    int stage = 0, slot = 0, nb = 0;
+    uint32_t phase = 0, uphase = 0, ph_e = 0;      // ph_e bit b: phase of acc_empty[b]
     bool ok = true;
     for (;;) {
       if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) { ok = false; break; }
@@ -263,9 +325,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
       if (u < 0) break;
       const Unit w = decode<EPI>(p, u);
-      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+      // a unit with a merged tail holds buffer 0 (full tile) and buffer 1 (tail, transposed)
+      const bool two = w.tail > 0;
+      const int acc = two ? 0 : nb;
+      if (!mbar_wait(&acc_empty[acc], ((ph_e >> acc) & 1u) ^ 1u, abort_flag, p.err)) { ok = false; break; }
+      ph_e ^= 1u << acc;
+      if (two) {
+        if (!mbar_wait(&acc_empty[1], ((ph_e >> 1) & 1u) ^ 1u, abort_flag, p.err)) { ok = false; break; }
+        ph_e ^= 2u;
+      }
+      nb = two ? 0 : nb ^ 1;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      const uint32_t d_tail = tmem_base + (uint32_t)BN;
+      // tail MMA: the weight block's two 128-column halves (MN-major, M = 128)
+      // against the tail rows (K-major, N = t16)
+      const uint32_t idesc_tail = idesc_bf16_f32(BM, w.t16 ? w.t16 : 16) | kIdescAMnMajor;
       for (int kb = 0; kb < w.nk; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
         uint8_t* a_st = sA + stage * A_BYTES;
@@ -293,16 +368,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                                               : sdesc_kmajor_sw128(a0 + k * UMMA_K * 2);
             tc_mma_bf16(d_tmem, ad, sdesc_mnmajor_sw128(b0 + k * UMMA_K * 128), IDESC, (kb | k) != 0);
           }
+          if (EPI != EPI_DW && two) {
+            const uint32_t t0 = smem_u32(sT + stage * T_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint64_t xd = sdesc_kmajor_sw128(t0 + k * UMMA_K * 2);
+              tc_mma_bf16(d_tail, sdesc_mnmajor_sw128(b0 + k * UMMA_K * 128), xd, idesc_tail, (kb | k) != 0);
+              tc_mma_bf16(d_tail + BN / 2, sdesc_mnmajor_sw128(b0 + 2 * MN_BOX_BYTES + k * UMMA_K * 128), xd,
+                          idesc_tail, (kb | k) != 0);
+            }
+          }
           tc_commit(&empty[stage]);
         }
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      if (lane == 0) tc_commit(&acc_full[acc]);     // with no k-block: arrives at once
+      if (lane == 0) {
+        tc_commit(&acc_full[acc]);                   // with no k-block: arrives at once
+        if (two) tc_commit(&acc_full[1]);
+      }
       __syncwarp();
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
     }
     if (lane == 0) {
       tc_commit(drain);
@@ -313,8 +399,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     // ---------------- epilogue (warps 2..5) ----------------
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
-    int acc = 0, slot = 0;
-    uint32_t acc_phase = 0, uphase = 0, stg_phase = 0;
+    int slot = 0, nb = 0;
+    uint32_t uphase = 0, stg_phase = 0, ph_f = 0;   // ph_f bit b: phase of acc_full[b]
     for (;;) {
       if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
       const int u = unit_ring[slot];
@@ -322,7 +408,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
       if (u < 0) break;
       const Unit w = decode<EPI>(p, u);
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.err)) break;
+      const bool two = w.tail > 0;                  // same buffer sequence as the MMA issuer
+      const int acc = two ? 0 : nb;
+      nb = two ? 0 : nb ^ 1;
+      if (!mbar_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err)) break;
+      ph_f ^= 1u << acc;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       if (EPI == EPI_DW) {
@@ -370,8 +460,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
           bulk_commit();
         }
         stg_phase ^= 1u;
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
         continue;
       } else {
         const int m = w.mt * BM + r;
@@ -426,8 +514,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (EPI != EPI_DW && two) {
+        // the merged tail (rows (mt + 1) * 128 ..), transposed in buffer 1
+        if (!mbar_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err)) break;
+        ph_f ^= 2u;
+        tc_fence_after();
+        epilogue_tail<EPI>(p, w, r, tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN);
+        tc_fence_before();
+        mbar_arrive(&acc_empty[1]);
+      }
     }
   }
 
@@ -505,6 +600,8 @@ static cudaError_t launch(const Params& p, int units, cudaStream_t st) {
 
 }  // namespace bwd
 
+int bwd_merge_rows() { return bwd::MERGE_ROWS; }
+
 cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st) {
   using namespace bwd;
   Params p{};
@@ -520,6 +617,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st) {
     // dA = dO W_d -> dU | dV (routed rows: dO = g dy; shared rows: dy itself)
     ok &= make_tmap(&p.a_r, a.dO_r, R, a.d, BM);
     ok &= make_tmap(&p.a_s, has_s ? a.dy : a.dO_r, has_s ? (uint64_t)a.T : R, a.d, BM);
+    ok &= make_tmap(&p.a32_r, a.dO_r, R, a.d, SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, has_s ? a.dy : a.dO_r, has_s ? (uint64_t)a.T : R, a.d, SUB_ROWS);
     ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, BK);
     ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, (uint64_t)(has_s ? a.E_s : a.E_r) * a.d, fs, BK);
     p.b1_r = p.b0_r; p.b1_s = p.b0_s;
@@ -539,6 +638,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st) {
     // dX = [dU | dV] [W_g ; W_u]
     ok &= make_tmap(&p.a_r, a.duv_r, R, 2 * (uint64_t)a.f_r, BM);
     ok &= make_tmap(&p.a_s, has_s ? a.duv_s : a.duv_r, RS, 2 * (uint64_t)fs, BM);
+    ok &= make_tmap(&p.a32_r, a.duv_r, R, 2 * (uint64_t)a.f_r, SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, has_s ? a.duv_s : a.duv_r, RS, 2 * (uint64_t)fs, SUB_ROWS);
     ok &= make_tmap(&p.b0_r, a.wg_r, (uint64_t)a.E_r * a.f_r, a.d, BK);
     ok &= make_tmap(&p.b1_r, a.wu_r, (uint64_t)a.E_r * a.f_r, a.d, BK);
     ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, (uint64_t)(has_s ? a.E_s : a.E_r) * fs, a.d, BK);

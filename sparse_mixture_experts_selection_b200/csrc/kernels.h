@@ -101,6 +101,7 @@ struct BwdArgs {
   int* err;
 };
 cudaError_t launch_bwd_tc(const BwdArgs& a, int which, cudaStream_t st);
+int bwd_merge_rows();   // backward dA / dX: tails of <= this many rows share the unit before
 
 // Backward of routing and combine (bf16 activations): per permuted row dO and
 // dL/dg; per token dz, dh; per expert de.
