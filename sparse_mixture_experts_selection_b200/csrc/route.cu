@@ -499,6 +499,57 @@ combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __r
   }
 }
 
+// Combine with K fixed at compile time: the K row indices stay in registers
+// and every row's 16-byte chunk is loaded before the sums, which run in the
+// same fixed order as combine_kernel (h, shared j ascending, slots k
+// ascending), so the results are bit-identical.
+template <typename T, int KT>
+__global__ void __launch_bounds__(128)
+combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
+                 const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int E_s,
+                 int add_residual, int n_slot_rows) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int t = blockIdx.x;
+  int rows[KT];
+#pragma unroll
+  for (int k = 0; k < KT; ++k) {
+    const int r = __ldg(row_of + (size_t)t * KT + k);
+    rows[k] = r < n_slot_rows ? r : -1;       // self-check: never read past the slot rows
+  }
+  for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * VEC; c < d; c += blockDim.x * gridDim.y * VEC) {
+    uint4 sv[KT];
+#pragma unroll
+    for (int k = 0; k < KT; ++k)
+      sv[k] = rows[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(slot + (size_t)rows[k] * d + c))
+                           : make_uint4(0, 0, 0, 0);
+    const uint4 hv = __ldg(reinterpret_cast<const uint4*>(h + (size_t)t * d + c));
+    float acc[VEC];
+    {
+      const T* v = reinterpret_cast<const T*>(&hv);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = add_residual ? to_f32(v[i]) : 0.f;
+    }
+    for (int j = 0; j < E_s; ++j) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(shared + ((size_t)j * n_tok + t) * d + c));
+      const T* v = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
+    }
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+      if (rows[k] < 0) continue;
+      const T* v = reinterpret_cast<const T*>(&sv[k]);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
+    }
+    uint4 out;
+    T* o = reinterpret_cast<T*>(&out);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) o[i] = from_f32<T>(acc[i]);
+    *reinterpret_cast<uint4*>(y + (size_t)t * d + c) = out;
+  }
+}
+
 // a9: b_i += gamma * sign(K*T - E_r*c_i) (one fp32 add), and MaxVio.
 __global__ void __launch_bounds__(1024)
 bias_update_kernel(const int* __restrict__ counts, float* __restrict__ b, float gamma,
@@ -759,7 +810,14 @@ void launch_combine(const void* h, const void* slot, const void* shared, const i
   const int max_split = (nvec + 127) / 128;
   split = split < 1 ? 1 : (split > max_split ? max_split : split);
   const dim3 grid(T, split);
-  if (dtype == MOE_DTYPE_BF16)
+  if (dtype == MOE_DTYPE_BF16 && (K == 2 || K == 4 || K == 6 || K == 8)) {
+    const bf16 *hh = (const bf16*)h, *sl = (const bf16*)slot, *sh = (const bf16*)shared;
+    bf16* yy = (bf16*)y;
+    if (K == 8) combine_k_kernel<bf16, 8><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+    else if (K == 6) combine_k_kernel<bf16, 6><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+    else if (K == 4) combine_k_kernel<bf16, 4><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+    else combine_k_kernel<bf16, 2><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+  } else if (dtype == MOE_DTYPE_BF16)
     combine_kernel<bf16><<<grid, 128, 0, st>>>((const bf16*)h, (const bf16*)slot, (const bf16*)shared,
                                             row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
   else
