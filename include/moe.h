@@ -265,6 +265,19 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
  *   are not used by this call).  Deterministic (no floating-point atomics).
  */
 /*
+ * Row gather for expert-parallel layouts (no counterpart step on the pages;
+ * the regrouping that an all-to-all dispatch needs, "Sparse Mixture-of-Experts
+ * ...", section 3 and "Mixture-of-Experts: Expert Parallelism, All-to-All
+ * Routing, ...", expert parallelism): dst[r] = src[map[r]] for r < n_rows, a
+ * zero row where map[r] < 0.  Rows are row_bytes long (a multiple of 4; src
+ * and dst 16-byte aligned when it is a multiple of 16).  map[r] >= n_src is
+ * reported through no error word here: the row is skipped (callers pass maps
+ * they built).  Enqueues one kernel; no host synchronisation.
+ */
+moe_status moe_gather_rows(const void* src, int64_t n_src, int32_t row_bytes, const int32_t* map,
+                           int64_t n_rows, void* dst, void* stream);
+
+/*
  * Backward of moe_layer_forward (train = 1): gradients of a loss L, given
  * dy = dL/dy [T, d] (bf16), with respect to h, the centroids e and every
  * expert weight, for the routing the forward chose.  The derivative of the

@@ -22,7 +22,7 @@ __all__ = [
     "moe_expert_ffn", "moe_expert_ffn_workspace_size", "moe_combine", "moe_bias_update",
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
     "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
-    "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3", "moe_layer_backward",
+    "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3", "moe_layer_backward", "moe_gather_rows",
     "moe_set_phase_events", "moe_selftest_bounded_wait",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
@@ -74,6 +74,7 @@ SIGNATURES = {
     "moe_quantized_bytes": (ctypes.c_int, [ctypes.c_int64, _I32, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_layer_backward": (ctypes.c_int, [_P] * 20 + [_P, ctypes.c_size_t, _P]),
     "moe_quantize_rows": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _I32, _P, _P]),
+    "moe_gather_rows": (ctypes.c_int, [_P, ctypes.c_int64, _I32, _P, ctypes.c_int64, _P, _P]),
     "moe_router_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "moe_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
@@ -167,6 +168,12 @@ def moe_router_stats_workspace_size(cfg: MoeConfig, seq_len: int = 0) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().moe_router_stats_workspace_size(ctypes.byref(cfg), int(seq_len), ctypes.byref(n)))
     return n.value
+
+
+def moe_gather_rows(src, n_src: int, row_bytes: int, map_, n_rows: int, dst, stream=None):
+    """dst[r] = src[map_[r]] row by row (zero where map_[r] < 0)."""
+    _check(lib().moe_gather_rows(_ptr(src), int(n_src), int(row_bytes), _ptr(map_), int(n_rows), _ptr(dst),
+                                 _stream(stream)))
 
 
 def moe_quantized_bytes(n_rows: int, cols: int) -> int:

@@ -654,6 +654,18 @@ moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* 
   return cuda_status();
 }
 
+moe_status moe_gather_rows(const void* src, int64_t n_src, int32_t row_bytes, const int32_t* map,
+                           int64_t n_rows, void* dst, void* stream) {
+  if (n_rows < 0 || n_src < 0) return fail(MOE_ERR_INVALID_ARG, "negative row count");
+  if (row_bytes < 4 || row_bytes % 4) return fail(MOE_ERR_INVALID_ARG, "row_bytes=%d must be a positive multiple of 4", row_bytes);
+  if (n_rows == 0) return MOE_OK;
+  MOE_NONNULL4(map);
+  if (row_bytes % 16 == 0) { MOE_NONNULL(dst); MOE_ALIGNED(src); } else { MOE_NONNULL4(dst); MOE_ALIGNED4(src); }
+  if (!src && n_src > 0) return fail(MOE_ERR_INVALID_ARG, "src is NULL");
+  moe::launch_gather_map(src, map, n_rows, n_src, row_bytes, dst, nullptr, static_cast<cudaStream_t>(stream));
+  return cuda_status();
+}
+
 moe_status moe_quantized_bytes(int64_t n_rows, int32_t cols, size_t* bytes) {
   if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
   if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows=%lld < 0", (long long)n_rows);

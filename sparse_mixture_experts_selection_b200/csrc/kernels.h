@@ -54,6 +54,8 @@ void launch_combine(const void* h, const void* slot, const void* shared, const i
                     int n_slot_rows, cudaStream_t st);
 void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
                         int T, cudaStream_t st);
+void launch_gather_map(const void* src, const int32_t* map, int64_t n_rows, int64_t n_src, int row_bytes,
+                       void* dst, int* err, cudaStream_t st);
 void launch_bounded_wait_selftest(uint64_t limit_ns, int* err, cudaStream_t st);
 // Tokens per partial sum of the per-sequence score means (router statistics).
 constexpr int kStatsChunk = 64;

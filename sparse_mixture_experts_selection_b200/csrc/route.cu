@@ -456,6 +456,31 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* _
   }
 }
 
+// dst[r] = src[map[r]] (map[r] < 0: a zero row) for r < n_rows; rows of
+// row_words 32-bit words, moved 16 bytes at a time when row_words % 4 == 0.
+__global__ void gather_map_kernel(const uint32_t* __restrict__ src, const int32_t* __restrict__ map,
+                                  int64_t n_rows, int64_t n_src, int row_words, uint32_t* __restrict__ dst,
+                                  int* err) {
+  const int lane = threadIdx.x % kWarp;
+  const int64_t nw = (int64_t)gridDim.x * blockDim.x / kWarp;
+  for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / kWarp; r < n_rows; r += nw) {
+    const int32_t m = map[r];
+    if (m >= n_src) {                                  // self-check: never read outside src
+      if (lane == 0 && err) set_device_error(err, MOE_DEVERR_INDEX);
+      continue;
+    }
+    uint32_t* d = dst + r * row_words;
+    if ((row_words & 3) == 0) {
+      uint4* d4 = reinterpret_cast<uint4*>(d);
+      const uint4* s4 = m >= 0 ? reinterpret_cast<const uint4*>(src + (int64_t)m * row_words) : nullptr;
+      for (int v = lane; v < row_words / 4; v += kWarp) d4[v] = s4 ? s4[v] : make_uint4(0, 0, 0, 0);
+    } else {
+      const uint32_t* s1 = m >= 0 ? src + (int64_t)m * row_words : nullptr;
+      for (int v = lane; v < row_words; v += kWarp) d[v] = s1 ? s1[v] : 0u;
+    }
+  }
+}
+
 // a8: y_t = res*h_t + sum_j shared[j,t] + sum_k slot[row_of[t,k]], fp32 in that order.
 template <typename T>
 __global__ void __launch_bounds__(128)
@@ -824,6 +849,14 @@ void launch_combine(const void* h, const void* slot, const void* shared, const i
     combine_kernel<float><<<grid, 128, 0, st>>>((const float*)h, (const float*)slot,
                                              (const float*)shared, row_of, (float*)y, T, d, K, E_s,
                                              add_residual, n_slot_rows);
+}
+
+void launch_gather_map(const void* src, const int32_t* map, int64_t n_rows, int64_t n_src, int row_bytes,
+                       void* dst, int* err, cudaStream_t st) {
+  if (n_rows <= 0) return;
+  const int64_t warps = n_rows < 148 * 64 ? n_rows : 148 * 64;
+  gather_map_kernel<<<(unsigned)((warps * kWarp + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint32_t*>(src), map, n_rows, n_src, row_bytes / 4, static_cast<uint32_t*>(dst), err);
 }
 
 void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
