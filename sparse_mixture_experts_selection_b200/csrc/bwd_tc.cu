@@ -193,6 +193,8 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all but the most recent bulk group have read their shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 
@@ -250,9 +252,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* stg_full = drain + 1;        // EPI_DW: the staged tile is complete (128 arrivals)
-  uint64_t* stg_free = stg_full + 1;     // EPI_DW: the previous tile's stores have read sOut
-  uint64_t* unit_full = stg_free + 1;
+  uint64_t* stg_full = drain + 1;        // EPI_DW [2]: a staged half tile is complete (128 arrivals)
+  uint64_t* stg_free = stg_full + 2;     // EPI_DW [2]: that buffer's previous stores have read it
+  uint64_t* unit_full = stg_free + 2;
   uint64_t* unit_empty = unit_full + UNIT_RING;
   volatile int* unit_ring = reinterpret_cast<volatile int*>(unit_empty + UNIT_RING);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UNIT_RING);
@@ -264,8 +266,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4 * kWarp); }
     for (int s = 0; s < UNIT_RING; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1 + 4 * kWarp); }
     mbar_init(drain, 1);
-    mbar_init(stg_full, 4 * kWarp);
-    mbar_init(stg_free, 1);
+    for (int q = 0; q < 2; ++q) { mbar_init(&stg_full[q], 4 * kWarp); mbar_init(&stg_free[q], 1); }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -400,7 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
     int slot = 0, nb = 0;
-    uint32_t uphase = 0, stg_phase = 0, ph_f = 0;   // ph_f bit b: phase of acc_full[b]
+    uint32_t uphase = 0, ph_f = 0;                 // ph_f bit b: phase of acc_full[b]
+    uint32_t stg_count = 0;                        // EPI_DW: half tiles staged so far
     for (;;) {
       if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
       const int u = unit_ring[slot];
@@ -416,50 +418,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       if (EPI == EPI_DW) {
-        // weight-gradient tile staged in sOut as four 128-row x 64-column boxes
-        // in the 128-byte swizzle layout the store map expects (16-byte chunk j
-        // of line r at chunk j ^ (r & 7)); this warp writes lines sub*32.. of
-        // each box, then one thread writes the four boxes by TMA stores that
-        // clip at the expert's M and N
+        // weight-gradient tile, written as two halves of 128 columns through
+        // two 32 KB staging buffers used in turn, so that one half's TMA stores
+        // drain while the next half is staged.  A half is two 128-row x
+        // 64-column boxes in the 128-byte swizzle layout of the store map
+        // (16-byte chunk j of line r at chunk j ^ (r & 7)); each warp writes
+        // lines sub*32.., one thread issues the stores, which clip at the
+        // expert's M and N
         const bool leader = warp == 2 && lane == 0;
-        if (leader) {
-          bulk_wait_read();                            // the previous tile's stores have read sOut
-          mbar_arrive(stg_free);
-        }
-        if (!mbar_wait(stg_free, stg_phase, abort_flag, p.err)) break;
+        bool aborted = false;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float dv[32];
-          tmem_ld32(tb + c, dv);
-          uint8_t* line = sOut + (c / 64) * (DW_OUT_BYTES / 4) + r * 128;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            if (w.nk == 0) pk = make_uint4(0, 0, 0, 0);        // an expert without rows
-            else {
-              pk.x = pack_bf16(dv[8 * v + 0], dv[8 * v + 1]);
-              pk.y = pack_bf16(dv[8 * v + 2], dv[8 * v + 3]);
-              pk.z = pack_bf16(dv[8 * v + 4], dv[8 * v + 5]);
-              pk.w = pack_bf16(dv[8 * v + 6], dv[8 * v + 7]);
-            }
-            const int chunk = ((c % 64) / 8 + v) ^ (r & 7);
-            *reinterpret_cast<uint4*>(line + chunk * 16) = pk;
+        for (int half = 0; half < 2; ++half) {
+          const int bf = stg_count & 1;
+          const uint32_t par = (stg_count >> 1) & 1u;
+          uint8_t* buf = sOut + bf * (DW_OUT_BYTES / 2);
+          if (leader) {
+            bulk_wait_read_1();                       // the stores that last used buf have read it
+            mbar_arrive(&stg_free[bf]);
           }
-        }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[acc]);                  // TMEM is free; the stores go on
-        fence_proxy_async_smem();
-        mbar_arrive(stg_full);
-        if (leader) {
-          if (!mbar_wait(stg_full, stg_phase, abort_flag, p.err)) break;
-          const int e = w.sh ? w.g - p.E_r : w.g;
-          const CUtensorMap* dm = w.sh ? &p.dws_s : &p.dws_r;
+          if (!mbar_wait(&stg_free[bf], par, abort_flag, p.err)) { aborted = true; break; }
+#pragma unroll 1
+          for (int c = 0; c < BN / 2; c += 32) {
+            float dv[32];
+            tmem_ld32(tb + half * (BN / 2) + c, dv);
+            uint8_t* line = buf + (c / 64) * (DW_OUT_BYTES / 4) + r * 128;
 #pragma unroll
-          for (int q = 0; q < BN / 64; ++q)
-            tma_store_3d(dm, sOut + q * (DW_OUT_BYTES / 4), w.nt * BN + q * 64, w.mt * BM, e);
-          bulk_commit();
+            for (int v = 0; v < 4; ++v) {
+              uint4 pk;
+              if (w.nk == 0) pk = make_uint4(0, 0, 0, 0);        // an expert without rows
+              else {
+                pk.x = pack_bf16(dv[8 * v + 0], dv[8 * v + 1]);
+                pk.y = pack_bf16(dv[8 * v + 2], dv[8 * v + 3]);
+                pk.z = pack_bf16(dv[8 * v + 4], dv[8 * v + 5]);
+                pk.w = pack_bf16(dv[8 * v + 6], dv[8 * v + 7]);
+              }
+              const int chunk = ((c % 64) / 8 + v) ^ (r & 7);
+              *reinterpret_cast<uint4*>(line + chunk * 16) = pk;
+            }
+          }
+          if (half == 1) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);              // TMEM is free; the stores go on
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&stg_full[bf]);
+          if (leader) {
+            if (!mbar_wait(&stg_full[bf], par, abort_flag, p.err)) { aborted = true; break; }
+            const int e = w.sh ? w.g - p.E_r : w.g;
+            const CUtensorMap* dm = w.sh ? &p.dws_s : &p.dws_r;
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              tma_store_3d(dm, buf + q * (DW_OUT_BYTES / 4), w.nt * BN + half * (BN / 2) + q * 64, w.mt * BM, e);
+            bulk_commit();
+          }
+          ++stg_count;
         }
-        stg_phase ^= 1u;
+        if (aborted) break;
         continue;
       } else {
         const int m = w.mt * BM + r;
