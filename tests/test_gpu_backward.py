@@ -97,6 +97,38 @@ def test_layer_backward_matches_oracle(name):
             _close(G[which][j], ref["grads"][(which, j)], (which, j))
 
 
+EDGE = {
+    "single_token": CASES["deepseek_small"].with_(T=1),
+    "dense_E1_K1": CASES["finegrained_near_tile"].with_(E_r=1, K=1),
+    "no_residual": CASES["finegrained_near_tile"].with_(add_residual=0),
+    # Zipf-skewed centroids: the hottest experts hold two full row tiles and a merged tail
+    "hot_expert": CASES["deepseek_small"].with_(T=700, centroid_skew="zipf_1.2"),
+    # more experts than selections: many experts without rows (zero weight gradients)
+    "sparse_experts": CASES["deepseek_small"].with_(T=40),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_layer_backward_edge_cases(name):
+    w = EDGE[name]
+    ref, dh, de, G = run_backward(w)
+    _close(dh, ref["dh"], "dh")
+    if np.any(ref["de"] != 0):
+        _close(de, ref["de"], "de")
+    else:                                   # one softmax expert: the gate is 1 whatever z is
+        assert np.max(np.abs(de)) <= 1e-6
+    for which in ("gate", "up", "down"):
+        for ex in range(w.E_r):
+            key = (which, ex)
+            if key in ref["grads"]:
+                _close(G[which][ex], ref["grads"][key], key)
+            else:
+                assert np.all(G[which][ex] == 0), key
+    for j in range(w.E_s):
+        for which in ("sgate", "sup", "sdown"):
+            _close(G[which][j], ref["grads"][(which, j)], (which, j))
+
+
 def test_backward_rejects_inference_config():
     w = CASES["deepseek_small"]
     cfg = moe.config_for(w)                                  # train = 0
