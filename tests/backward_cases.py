@@ -1,0 +1,91 @@
+"""Workloads and the parity bar of the layer-backward tests (shared by the GPU
+parity test and the CPU test that derives the bar from the bf16 storage model).
+
+Bar, per tensor (per expert for weight gradients), got against the oracle's
+float64 gradients ref:
+  normwise    ||got - ref|| <= NORM_TOL * ||ref||
+  elementwise max(|got - ref| - 2^-8 |ref|) <= ELEM_TOL * RMS(ref)
+the 2^-8 |ref| term allowing the stored bf16 value's own rounding.  The bf16
+storage model of the backward (bf16_backward_model) sits at most at 0.0082
+normwise and 0.108 elementwise from the oracle on these cases (one token's dL/de
+and few-row experts' weight gradients, outer products of a handful of rows,
+carry the heaviest elementwise tails); the bars leave room above that."""
+import numpy as np
+
+import moe_inputs as mi
+from oracle import moe_oracle as mo
+
+NORM_TOL = 2e-2
+ELEM_TOL = 0.15
+
+W = mi.WORKLOADS
+CASES = {
+    "deepseek_small": W["deepseek_v3"].with_(T=520, d_model=256, E_r=64, E_s=1, K=6, d_ffn=256,
+                                             d_ffn_shared=384, n_groups=8, topk_groups=3),
+    "finegrained_near_tile": W["finegrained_64x1408"].with_(T=440, d_model=192, E_r=16, E_s=2, K=4,
+                                                           d_ffn=192, d_ffn_shared=128),
+    # capacity 1.0: some (token, expert) pairs are dropped
+    "finegrained_cf": W["finegrained_64x1408_cf1.25"].with_(T=600, d_model=192, E_r=16, E_s=2, K=4,
+                                                            d_ffn=192, d_ffn_shared=128, capacity_factor=1.0),
+    "mixtral_small": W["mixtral_8x14336"].with_(T=300, d_model=256, d_ffn=320),
+}
+EDGE = {
+    "single_token": CASES["deepseek_small"].with_(T=1),
+    "dense_E1_K1": CASES["finegrained_near_tile"].with_(E_r=1, K=1),
+    "no_residual": CASES["finegrained_near_tile"].with_(add_residual=0),
+    # Zipf-skewed centroids: the hottest experts hold two full row tiles and a merged tail
+    "hot_expert": CASES["deepseek_small"].with_(T=700, centroid_skew="zipf_1.2"),
+    # more experts than selections: many experts without rows (zero weight gradients)
+    "sparse_experts": CASES["deepseek_small"].with_(T=40),
+}
+
+
+def inputs(w, seed=7):
+    """h, e, b, the oracle's fp32 scores s, its routing (idx, gates, disp) and a
+    bf16 output gradient dy of workload w."""
+    from gpu_helpers import oracle_cfg
+    h, e, b = mi.gen_h(w, 0), mi.gen_centroids(w), mi.gen_bias(w)
+    cfg = oracle_cfg(w)
+    s = mo.affinity(h, e, w.score_fn)
+    b_sel = b if w.score_fn == 0 else np.zeros(w.E_r, np.float32)
+    idx, gates, disp = mo.route(cfg, s, b_sel)
+    rng = np.random.default_rng(seed)
+    dy = mi.round_bf16(rng.normal(size=(w.T, w.d_model)).astype(np.float32))
+    return cfg, h, e, b, s, idx, gates, disp, dy
+
+
+def errors(got, ref):
+    """(normwise, elementwise) errors of got against ref as fractions of the bar's
+    scales (||ref||, RMS(ref))."""
+    ref = np.asarray(ref, np.float64)
+    got = np.asarray(got, np.float64)
+    if ref.size == 0:
+        return 0.0, 0.0
+    nref = np.linalg.norm(ref)
+    scale = np.sqrt(np.mean(ref ** 2))
+    if nref == 0.0:
+        return float(np.max(np.abs(got))), float(np.max(np.abs(got)))
+    return (float(np.linalg.norm(got - ref) / nref),
+            float(np.max(np.abs(got - ref) - 2.0 ** -8 * np.abs(ref)) / scale))
+
+
+def check(got, ref, what):
+    got = np.asarray(got, np.float64)
+    assert np.all(np.isfinite(got)), what
+    n, m = errors(got, ref)
+    assert n <= NORM_TOL and m <= ELEM_TOL, (what, n, m)
+
+
+def each_gradient(w, ref, G):
+    """(what, got, ref) for every weight gradient; experts without kept rows
+    have no entry in ref and must get exactly zero (checked here)."""
+    for which in ("gate", "up", "down"):
+        for ex in range(w.E_r):
+            key = (which, ex)
+            if key in ref["grads"]:
+                yield key, G[which][ex], ref["grads"][key]
+            else:
+                assert np.all(G[which][ex] == 0), key
+    for j in range(w.E_s):
+        for which in ("sgate", "sup", "sdown"):
+            yield (which, j), G[which][j], ref["grads"][(which, j)]
