@@ -94,8 +94,8 @@ Layout make_layout(const moe_config& c) {
   L.slot_r = take((size_t)L.R * c.d_model * es);
   L.slot_s = take((size_t)c.E_s * c.T * c.d_model * es);
   L.xs = take(q8 ? (size_t)L.R * 4 : 0);
-  L.hq = take(q8 && c.E_s ? (size_t)c.T * c.d_model : 0);
-  L.hs = take(q8 && c.E_s ? (size_t)c.T * 4 : 0);
+  L.hq = take(q8 ? (size_t)c.T * c.d_model : 0);
+  L.hs = take(q8 ? (size_t)c.T * 4 : 0);
   L.actq_r = take(q8 ? (size_t)L.R * c.d_ffn : 0);
   L.actq_s = take(q8 ? (size_t)c.E_s * c.T * fs : 0);
   L.as_r = take(q8 ? (size_t)L.R * 4 : 0);
@@ -469,13 +469,12 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   void* x_perm = at<void>(ws, L.x_perm);
   const bool q8 = is_q8(c.dtype);
   if (q8) {
-    // gather + quantize: e4m3 rows of x_perm with their scales, and of h for
-    // the shared experts
-    moe::launch_quantize_rows(h, MOE_DTYPE_BF16, perm_tok, c.T, offsets + c.E_r, L.R, c.d_model,
-                              static_cast<uint8_t*>(x_perm), at<float>(ws, L.xs), err, st);
-    if (c.E_s)
-      moe::launch_quantize_rows(h, MOE_DTYPE_BF16, nullptr, 0, nullptr, c.T, c.d_model,
-                                at<uint8_t>(ws, L.hq), at<float>(ws, L.hs), err, st);
+    // quantize each token's row of h once (the shared experts' input), then
+    // gather the e4m3 rows and their scales into expert order
+    moe::launch_quantize_rows(h, MOE_DTYPE_BF16, nullptr, 0, nullptr, c.T, c.d_model,
+                              at<uint8_t>(ws, L.hq), at<float>(ws, L.hs), err, st);
+    moe::launch_gather(at<uint8_t>(ws, L.hq), perm_tok, offsets + c.E_r, x_perm, c.d_model, 1, (int)L.R,
+                       c.T, err, st, at<float>(ws, L.hs), at<float>(ws, L.xs));
   } else {
     moe::launch_gather(h, perm_tok, offsets + c.E_r, x_perm, c.d_model, (int)es, (int)L.R, c.T, err, st);
   }
@@ -498,9 +497,9 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
   if (c.train) { a.uv_r = at<void>(ws, L.uv_r); a.uv_s = c.E_s ? at<void>(ws, L.uv_s) : a.uv_r; }
   if (q8) {
     a.q8 = 1;
-    a.x_s = c.E_s ? at<void>(ws, L.hq) : x_perm;
+    a.x_s = at<void>(ws, L.hq);
     a.xs_r = at<float>(ws, L.xs);
-    a.xs_s = c.E_s ? at<float>(ws, L.hs) : a.xs_r;
+    a.xs_s = at<float>(ws, L.hs);
     a.actq_r = at<void>(ws, L.actq_r); a.actq_s = c.E_s ? at<void>(ws, L.actq_s) : a.actq_r;
     a.as_r = at<float>(ws, L.as_r); a.as_s = c.E_s ? at<float>(ws, L.as_s) : a.as_r;
   }

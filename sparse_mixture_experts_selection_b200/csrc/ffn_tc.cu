@@ -31,7 +31,9 @@
 // weight tile, which feeds both the normal MMA and the transposed tail MMA.
 // Experts of a little more than 128 tokens -- the common case when T*K/E_r is
 // near 128 -- thus stream their weights through shared memory once, not twice,
-// and spend no MMAs on padding.  Such a unit holds both TMEM accumulators.
+// and spend no MMAs on padding.  Such a unit holds both TMEM accumulators; its
+// epilogue drains the short tail first and the next unit takes the tail's
+// buffer, so only the unit before it waits for a whole epilogue.
 #include <algorithm>
 #include <cuda.h>
 #include "common.cuh"
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           if (!mbar_wait(&acc_empty[1], ((ph_e >> 1) & 1u) ^ 1u, abort_flag, p.err)) break;
           ph_e ^= 2u;
         }
-        nb = two ? 0 : nb ^ 1;
+        nb = two ? 1 : nb ^ 1;              // after a merged unit, the tail's buffer frees first
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         const uint32_t d_tail = tmem_base + (uint32_t)BN;
@@ -471,10 +473,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       uint16_t* out = (sh ? p.out_s : p.out_r) + orow * ncols;
       const bool two = w.tail > 0;
       const int acc = two ? 0 : nb;
-      nb = two ? 0 : nb ^ 1;
-      if (!mbar_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err)) break;
-      ph_f ^= 1u << acc;
-      tc_fence_after();
+      nb = two ? 1 : nb ^ 1;
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       // transposed tiles: this thread owns output column(s) r of the unit and
       // walks the rows along the accumulator columns
@@ -496,6 +495,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       // training forward: U | V rows of this tile (row 0 of the tile)
       uint16_t* uv0 = (EPI == EPI_SWIGLU && (sh ? p.uv_s : p.uv_r))
                           ? (sh ? p.uv_s : p.uv_r) + row0 * (size_t)(2 * ncols) : nullptr;
+      if (EPI != EPI_ROUTER && two) {
+        // the merged tail (rows (mt + 1) * 128 .. + tail, transposed, buffer 1)
+        // first: its buffer is the one the next unit takes
+        if (!mbar_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err)) break;
+        ph_f ^= 2u;
+        tc_fence_after();
+        epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
+                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
+                                 xs ? xs + BM : nullptr, wsA, wsB, uv0 ? uv0 + (size_t)BM * 2 * ncols : nullptr);
+        tc_fence_before();
+        mbar_arrive(&acc_empty[1]);
+      }
+      if (!mbar_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err)) break;
+      ph_f ^= 1u << acc;
+      tc_fence_after();
       if (EPI != EPI_ROUTER && w.n16) {
         epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb,
                                  xs, wsA, wsB, uv0);
@@ -589,17 +603,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      if (EPI != EPI_ROUTER && two) {
-        // the merged tail: rows (mt + 1) * 128 .. + tail, transposed, in buffer 1
-        if (!mbar_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err)) break;
-        ph_f ^= 2u;
-        tc_fence_after();
-        epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
-                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
-                                 xs ? xs + BM : nullptr, wsA, wsB, uv0 ? uv0 + (size_t)BM * 2 * ncols : nullptr);
-        tc_fence_before();
-        mbar_arrive(&acc_empty[1]);
-      }
     }
   }
 

@@ -47,8 +47,11 @@ void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int merg
 void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
                     const int* chunk_base, int cap, int T, int K, int E, int32_t* perm_tok,
                     int32_t* row_of, float* row_gate, int* err, cudaStream_t st);
+// x_perm[r] = h[perm_tok[r]] (rows of d * elem_bytes bytes, a multiple of 16)
+// for r < *n_rows_ptr; with s_src also s_dst[r] = s_src[perm_tok[r]]
 void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
-                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st);
+                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st,
+                   const float* s_src = nullptr, float* s_dst = nullptr);
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
                     void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
                     int n_slot_rows, cudaStream_t st);

@@ -430,10 +430,12 @@ scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gates,
   }
 }
 
-// x_perm[r] = h[perm_tok[r]] for r < offsets[E] (one warp per row, 16-byte moves)
+// x_perm[r] = h[perm_tok[r]] for r < offsets[E] (one warp per row, 16-byte
+// moves); with s_src, also s_dst[r] = s_src[perm_tok[r]] (row scales of e4m3 rows)
 __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* __restrict__ perm_tok,
                                    const int* __restrict__ n_rows_ptr, uint4* __restrict__ x_perm,
-                                   int vec_per_row, int n_tok, int max_rows, int* err) {
+                                   int vec_per_row, int n_tok, int max_rows, int* err,
+                                   const float* __restrict__ s_src, float* __restrict__ s_dst) {
   const int n = min(*n_rows_ptr, max_rows);
   const int lane = threadIdx.x % kWarp;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
@@ -444,6 +446,7 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* _
       if (lane == 0) set_device_error(err, MOE_DEVERR_INDEX);
       continue;
     }
+    if (s_src && lane == 0) s_dst[r] = s_src[t];
     const uint4* src = h + (size_t)t * vec_per_row;
     uint4* dst = x_perm + (size_t)r * vec_per_row;
     // 4 independent 16-byte loads in flight per lane before the stores
@@ -817,13 +820,14 @@ void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
 }
 
 void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
-                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st) {
+                   int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st,
+                   const float* s_src, float* s_dst) {
   int vec = d * elem_bytes / 16;
   int warps = max_rows < 148 * 64 ? max_rows : 148 * 64;
   if (warps < 1) warps = 1;
   int blocks = (warps * 32 + 255) / 256;
   gather_rows_kernel<<<blocks, 256, 0, st>>>((const uint4*)h, perm_tok, n_rows_ptr, (uint4*)x_perm,
-                                             vec, n_tok, max_rows, err);
+                                             vec, n_tok, max_rows, err, s_src, s_dst);
 }
 
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
