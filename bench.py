@@ -261,6 +261,30 @@ def train_work(w, kept: np.ndarray):
     return flops, nbytes
 
 
+def train_writes(w) -> int:
+    """Bytes one backward writes: every weight gradient (routed and shared,
+    bf16), dh (bf16) and de (fp32)."""
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    return w.E_r * 3 * d * f * 2 + w.E_s * 3 * d * fs * 2 + w.T * d * 2 + w.E_r * d * 4
+
+
+def measure_write_gbs(torch, dev, nbytes=4 << 30, reps=5) -> float:
+    """HBM write-only bandwidth on this GPU now: a device fill of nbytes timed
+    with CUDA events (a denominator for write-bound kernels, not our work)."""
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        buf.fill_(1)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        buf.fill_(1)
+    b.record()
+    torch.cuda.synchronize()
+    gbs = reps * nbytes / (a.elapsed_time(b) * 1e-3) / 1e9
+    del buf
+    return gbs
+
+
 def run_train(args, w, rank, world, local_rank):
     """Training step: moe_layer_forward (train = 1) + moe_layer_backward."""
     import torch
@@ -345,6 +369,11 @@ def run_train(args, w, rank, world, local_rank):
     b_flops, b_bytes = float(np.mean([x[0] for x in tw])), float(np.mean([x[1] for x in tw]))
     bwd_s = float(np.mean(bwd)) / 1000
     t_roof_b = max(b_flops / (bf16_peak * 1e12), b_bytes / (hbm * 1e9))
+    # the weight-gradient launches only write (their operands are L2-resident):
+    # they are bounded by the write-only bandwidth, which is well below the copy figure
+    write_gbs = measure_write_gbs(torch, dev)
+    b_writes = float(train_writes(w))
+    t_roof_w = max(b_flops / (bf16_peak * 1e12), (b_bytes - b_writes) / (hbm * 1e9) + b_writes / (write_gbs * 1e9))
     ms_per_step = elapsed_ms / args.steps
     line = {
         "metric": "MoE-layer training step (forward + backward) tokens/s", "value": job_throughput(world, w.T, args.steps, elapsed_ms),
@@ -358,7 +387,11 @@ def run_train(args, w, rank, world, local_rank):
                               "flops": b_flops, "bytes": b_bytes,
                               "bound": "hbm" if b_bytes / (hbm * 1e9) >= b_flops / (bf16_peak * 1e12) else "tensor",
                               "achieved_gbs": b_bytes / bwd_s / 1e9, "achieved_tflops": b_flops / bwd_s / 1e12,
-                              "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained"},
+                              "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained",
+                              "write_aware": {"t_roof_ms": 1000 * t_roof_w, "frac": 1000 * t_roof_w / float(np.mean(bwd)),
+                                              "writes": b_writes, "write_gbs": write_gbs,
+                                              "note": "writes at the write-only bandwidth measured live "
+                                                      "(device fill), reads at the copy figure"}},
         "clocks": clk,
         # forward 11 + backward: groups, (sigmoid: scan + scatter of every selected
         # pair), 2 tail zeroings, rows, 5 GEMMs, gates, dh, de
