@@ -268,21 +268,22 @@ def train_writes(w) -> int:
     return w.E_r * 3 * d * f * 2 + w.E_s * 3 * d * fs * 2 + w.T * d * 2 + w.E_r * d * 4
 
 
-def measure_write_gbs(torch, dev, nbytes=4 << 30, reps=5) -> float:
-    """HBM write-only bandwidth on this GPU now: a device fill of nbytes timed
-    with CUDA events (a denominator for write-bound kernels, not our work)."""
+def measure_write_gbs(torch, dev, nbytes=4 << 30, reps=6) -> float:
+    """HBM write-only bandwidth on this GPU now: the fastest of `reps` device
+    fills of nbytes, each timed with CUDA events (a denominator for
+    write-bound kernels, not our work)."""
     buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    for _ in range(3):
-        buf.fill_(1)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
+    buf.fill_(1)
+    best = 0.0
     for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
         buf.fill_(1)
-    b.record()
-    torch.cuda.synchronize()
-    gbs = reps * nbytes / (a.elapsed_time(b) * 1e-3) / 1e9
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
     del buf
-    return gbs
+    return best
 
 
 def run_train(args, w, rank, world, local_rank):

@@ -48,14 +48,29 @@ bwd_rows_kernel(const uint16_t* __restrict__ dy, const int32_t* __restrict__ per
     const uint16_t* sr = slot + (size_t)r * d;
     uint16_t* out = dO + (size_t)r * d;
     float acc = 0.0f;
-    for (int c = lane * 8; c < d; c += kWarp * 8) {
-      float a[8], b[8];
-      unpack8(*reinterpret_cast<const uint4*>(dyr + c), a);
-      unpack8(*reinterpret_cast<const uint4*>(sr + c), b);
+    // four 16-byte vectors of dy and of the slot in flight per lane; the
+    // products are accumulated in column order
+    constexpr int U = 4;
+    for (int c0 = lane * 8; c0 < d; c0 += U * kWarp * 8) {
+      uint4 qa[U], qb[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(a[i], b[i], acc);
-      *reinterpret_cast<uint4*>(out + c) = make_uint4(pack2(g * a[0], g * a[1]), pack2(g * a[2], g * a[3]),
-                                                       pack2(g * a[4], g * a[5]), pack2(g * a[6], g * a[7]));
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kWarp * 8;
+        qa[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(dyr + c)) : make_uint4(0, 0, 0, 0);
+        qb[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(sr + c)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kWarp * 8;
+        if (c >= d) break;
+        float a[8], b[8];
+        unpack8(qa[u], a);
+        unpack8(qb[u], b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc = fmaf(a[i], b[i], acc);
+        *reinterpret_cast<uint4*>(out + c) = make_uint4(pack2(g * a[0], g * a[1]), pack2(g * a[2], g * a[3]),
+                                                         pack2(g * a[4], g * a[5]), pack2(g * a[6], g * a[7]));
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
@@ -114,41 +129,57 @@ bwd_gate_kernel(const float* __restrict__ s, const int32_t* __restrict__ idx,
   }
 }
 
-// One block per token: dh = a dy + sum_j dX^S_j + sum_{k kept} dX_row + sum_i dz_i e_i.
-__global__ void __launch_bounds__(256)
+// dh = a dy + sum_j dX^S_j + sum_{k kept} dX_row + sum_i dz_i e_i: block
+// (t, y) covers 8-column vectors y*128 + tid, += 128 * gridDim.y of token t.
+// The K routed rows are loaded KC at a time before they are added, so their
+// loads are in flight together; the sums keep the order above.
+constexpr int kDhChunk = 8;
+__global__ void __launch_bounds__(128)
 bwd_dh_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ dx_r,
               const uint16_t* __restrict__ dx_s, const int32_t* __restrict__ row_of,
               const float* __restrict__ dz, const float* __restrict__ e, const int32_t* __restrict__ idx,
               int T, int d, int K, int E, int E_s, int add_residual, int n_rows, int sparse,
               uint16_t* __restrict__ dh) {
   const int t = blockIdx.x;
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+  const int nvec = d / 8;
+  for (int v0 = blockIdx.y * blockDim.x + threadIdx.x; v0 < nvec; v0 += blockDim.x * gridDim.y) {
+    const int c = v0 * 8;
     float acc[8], v[8];
-    unpack8(*reinterpret_cast<const uint4*>(dy + (size_t)t * d + c), v);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(dy + (size_t)t * d + c)), v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = add_residual ? v[i] : 0.0f;
     for (int j = 0; j < E_s; ++j) {
-      unpack8(*reinterpret_cast<const uint4*>(dx_s + ((size_t)j * T + t) * d + c), v);
+      unpack8(__ldg(reinterpret_cast<const uint4*>(dx_s + ((size_t)j * T + t) * d + c)), v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += v[i];
     }
-    for (int k = 0; k < K; ++k) {
-      const int ro = row_of[(size_t)t * K + k];
-      if (ro < 0 || ro >= n_rows) continue;
-      unpack8(*reinterpret_cast<const uint4*>(dx_r + (size_t)ro * d + c), v);
+    for (int k0 = 0; k0 < K; k0 += kDhChunk) {
+      uint4 xr[kDhChunk];
+      bool ok[kDhChunk];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      for (int q = 0; q < kDhChunk; ++q) {
+        const int ro = k0 + q < K ? __ldg(row_of + (size_t)t * K + k0 + q) : -1;
+        ok[q] = ro >= 0 && ro < n_rows;
+        xr[q] = ok[q] ? __ldg(reinterpret_cast<const uint4*>(dx_r + (size_t)ro * d + c)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int q = 0; q < kDhChunk; ++q) {
+        if (!ok[q]) continue;
+        unpack8(xr[q], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      }
     }
     // router term: sigmoid routing has dz != 0 only on the K selected experts
     // (ascending, as idx stores them); softmax touches every expert
     const float* zr = dz + (size_t)t * E;
     const int nj = sparse ? K : E;
     for (int q = 0; q < nj; ++q) {
-      const int j = sparse ? idx[(size_t)t * K + q] : q;
-      const float z = zr[j];
+      const int j = sparse ? __ldg(idx + (size_t)t * K + q) : q;
+      const float z = __ldg(zr + j);
       if (z == 0.0f) continue;
-      const float4 e0 = *reinterpret_cast<const float4*>(e + (size_t)j * d + c);
-      const float4 e1 = *reinterpret_cast<const float4*>(e + (size_t)j * d + c + 4);
+      const float4 e0 = __ldg(reinterpret_cast<const float4*>(e + (size_t)j * d + c));
+      const float4 e1 = __ldg(reinterpret_cast<const float4*>(e + (size_t)j * d + c + 4));
       acc[0] = fmaf(z, e0.x, acc[0]); acc[1] = fmaf(z, e0.y, acc[1]);
       acc[2] = fmaf(z, e0.z, acc[2]); acc[3] = fmaf(z, e0.w, acc[3]);
       acc[4] = fmaf(z, e1.x, acc[4]); acc[5] = fmaf(z, e1.y, acc[5]);
@@ -159,39 +190,49 @@ bwd_dh_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ dx_r
   }
 }
 
-// de [E, d] = dz^T h: one block per (expert, 256 columns), tokens in order.
-__global__ void __launch_bounds__(256)
-bwd_de_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ h, int T, int d, int E,
-              float* __restrict__ de) {
+// de [E, d] = dz^T h, tokens in ascending order: block (j, y) covers 8-column
+// vectors y*128 + tid of expert j.  SPARSE (sigmoid routing): dz is non-zero
+// only on the selected pairs, and the pairs of expert j (every selected
+// (t, j), dropped ones included) are rows sel_off[j] .. sel_off[j+1] of
+// sel_tok in ascending token order; otherwise every token.  Four tokens'
+// rows are loaded before they are accumulated (in order).
+constexpr int kDeUnroll = 4;
+template <bool SPARSE>
+__global__ void __launch_bounds__(128)
+bwd_de_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ h, const int32_t* __restrict__ sel_tok,
+              const int* __restrict__ sel_off, int T, int d, int E, float* __restrict__ de) {
   const int j = blockIdx.x;
-  const int c = blockIdx.y * blockDim.x + threadIdx.x;
-  float acc = 0.0f;
-  for (int t = 0; t < T; ++t) {
-    const float z = __ldg(dz + (size_t)t * E + j);
-    if (z == 0.0f) continue;
-    if (c < d) acc = fmaf(z, __uint_as_float((uint32_t)h[(size_t)t * d + c] << 16), acc);
+  const int vi = blockIdx.y * blockDim.x + threadIdx.x;
+  if (vi >= d / 8) return;
+  const int c = vi * 8;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  const int r0 = SPARSE ? __ldg(sel_off + j) : 0;
+  const int r1 = SPARSE ? __ldg(sel_off + j + 1) : T;
+  for (int r = r0; r < r1; r += kDeUnroll) {
+    float z[kDeUnroll];
+    uint4 hv[kDeUnroll];
+#pragma unroll
+    for (int u = 0; u < kDeUnroll; ++u) {
+      int t = r + u < r1 ? (SPARSE ? __ldg(sel_tok + r + u) : r + u) : -1;
+      if (t >= T) t = -1;
+      z[u] = t >= 0 ? __ldg(dz + (size_t)t * E + j) : 0.0f;
+      hv[u] = (t >= 0 && z[u] != 0.0f) ? __ldg(reinterpret_cast<const uint4*>(h + (size_t)t * d + c))
+                                       : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kDeUnroll; ++u) {
+      if (z[u] == 0.0f) continue;
+      float v[8];
+      unpack8(hv[u], v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(z[u], v[i], acc[i]);
+    }
   }
-  if (c < d) de[(size_t)j * d + c] = acc;
-}
-
-// de for sigmoid routing: dz is non-zero only on the selected pairs; the
-// pairs of expert j (every selected (t, j), dropped ones included) are rows
-// sel_off[j] .. sel_off[j+1] of sel_tok, in ascending token order.
-__global__ void __launch_bounds__(256)
-bwd_de_sparse_kernel(const float* __restrict__ dz, const uint16_t* __restrict__ h,
-                     const int32_t* __restrict__ sel_tok, const int* __restrict__ sel_off, int T, int d,
-                     int E, float* __restrict__ de) {
-  const int j = blockIdx.x;
-  const int c = blockIdx.y * blockDim.x + threadIdx.x;
-  float acc = 0.0f;
-  const int r0 = sel_off[j], r1 = sel_off[j + 1];
-  for (int r = r0; r < r1; ++r) {
-    const int t = sel_tok[r];
-    if (t < 0 || t >= T) continue;
-    const float z = __ldg(dz + (size_t)t * E + j);
-    if (c < d) acc = fmaf(z, __uint_as_float((uint32_t)h[(size_t)t * d + c] << 16), acc);
-  }
-  if (c < d) de[(size_t)j * d + c] = acc;
+  float4* out = reinterpret_cast<float4*>(de + (size_t)j * d + c);
+  out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
 // Zero rows n .. n+63 (n = *n_rows_ptr, capped at max_rows) of a bf16 [max_rows, cols]
@@ -222,13 +263,17 @@ void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st) {
 void launch_bwd_gate_dh_de(const BwdRouteArgs& a, cudaStream_t st) {
   bwd_gate_kernel<<<(a.T + 7) / 8, 256, 0, st>>>(a.s, a.idx, a.row_of, a.dg_row, a.score_fn, a.T, a.E, a.K, a.dz);
   const int sparse = a.score_fn == 0;
-  bwd_dh_kernel<<<a.T, 256, 0, st>>>(a.dy, a.dx_r, a.dx_s, a.row_of, a.dz, a.e, a.idx, a.T, a.d, a.K, a.E,
-                                     a.E_s, a.add_residual, a.max_rows, sparse, a.dh);
+  const int nvec = a.d / 8;
+  int split = (2 * 148 + a.T - 1) / a.T;                // fill the GPU for short batches
+  const int max_split = (nvec + 127) / 128;
+  split = split < 1 ? 1 : (split > max_split ? max_split : split);
+  bwd_dh_kernel<<<dim3(a.T, split), 128, 0, st>>>(a.dy, a.dx_r, a.dx_s, a.row_of, a.dz, a.e, a.idx, a.T, a.d, a.K,
+                                                 a.E, a.E_s, a.add_residual, a.max_rows, sparse, a.dh);
+  const dim3 g_de(a.E, (nvec + 127) / 128);
   if (sparse)
-    bwd_de_sparse_kernel<<<dim3(a.E, (a.d + 255) / 256), 256, 0, st>>>(a.dz, a.h, a.sel_tok, a.sel_off, a.T,
-                                                                       a.d, a.E, a.de);
+    bwd_de_kernel<true><<<g_de, 128, 0, st>>>(a.dz, a.h, a.sel_tok, a.sel_off, a.T, a.d, a.E, a.de);
   else
-    bwd_de_kernel<<<dim3(a.E, (a.d + 255) / 256), 256, 0, st>>>(a.dz, a.h, a.T, a.d, a.E, a.de);
+    bwd_de_kernel<false><<<g_de, 128, 0, st>>>(a.dz, a.h, nullptr, nullptr, a.T, a.d, a.E, a.de);
 }
 
 }  // namespace moe
