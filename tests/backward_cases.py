@@ -37,6 +37,8 @@ EDGE = {
     "hot_expert": CASES["deepseek_small"].with_(T=700, centroid_skew="zipf_1.2"),
     # more experts than selections: many experts without rows (zero weight gradients)
     "sparse_experts": CASES["deepseek_small"].with_(T=40),
+    # softmax routing with capacity 1.0: 34 of the 600 pairs dropped (dz reaches every expert)
+    "softmax_dropped": CASES["mixtral_small"].with_(capacity_factor=1.0),
 }
 
 

@@ -23,7 +23,7 @@ def _both(w):
 
 
 @pytest.mark.parametrize("name", ["deepseek_small", "single_token", "hot_expert", "sparse_experts",
-                                  "finegrained_cf", "dense_E1_K1"])
+                                  "finegrained_cf", "dense_E1_K1", "softmax_dropped"])
 def test_bf16_model_within_three_quarters_of_the_bar(name):
     w = ALL[name]
     ref, model = _both(w)

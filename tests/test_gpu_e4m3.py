@@ -28,6 +28,10 @@ SMALL_E4M3 = {
     "finegrained_near_tile_e4m3": W["finegrained_64x1408"].with_(
         T=440, d_model=192, E_r=16, E_s=2, K=4, d_ffn=192, d_ffn_shared=144, dtype="bf16_e4m3"),
     "mixtral_small_e4m3": W["mixtral_8x14336"].with_(T=300, d_model=256, d_ffn=320, dtype="bf16_e4m3"),
+    # capacity 1.0: 99 of the 1760 (token, expert) pairs are dropped
+    "finegrained_cf_e4m3": W["finegrained_64x1408"].with_(
+        T=440, d_model=192, E_r=16, E_s=2, K=4, d_ffn=192, d_ffn_shared=128, capacity_factor=1.0,
+        dtype="bf16_e4m3"),
     "decode_small_e4m3": W["deepseek_v3_decode_e4m3"].with_(T=24, d_model=320, E_r=64, d_ffn=128,
                                                             d_ffn_shared=128, topk_groups=4),
 }
