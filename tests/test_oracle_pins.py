@@ -271,9 +271,158 @@ def pin_permutation_properties(seed=9):
     assert (0, 0) in kept_fwd and (0, 0) not in kept_rev
 
 
+def _brute_gaps(key, K, n_groups=1, topk_groups=1, topn=0):
+    """Both gaps of one token by enumeration: the kept groups are the one
+    subset whose every member beats every non-member; the selected experts
+    likewise among the eligible ones.  Returns (top-K gap, group gap): the
+    smallest selected key minus the largest eligible unselected key, and the
+    smallest kept group score minus the largest dropped one (inf when there is
+    nothing to compare)."""
+    E = len(key)
+    gs = E // n_groups
+    group_gap = math.inf
+    if n_groups > 1 and topn > 0:
+        elig = _brute_groups(key, n_groups, topk_groups, topn)
+        G = []
+        for g in range(n_groups):
+            vals = sorted(key[g * gs:(g + 1) * gs], reverse=True)[:topn]
+            acc = F32(vals[0])
+            for v in vals[1:]:
+                acc = F32(acc + F32(v))
+            G.append(float(acc))
+        kept_g = {i // gs for i in range(E) if elig[i]}
+        dropped_g = [G[g] for g in range(n_groups) if g not in kept_g]
+        if dropped_g:
+            group_gap = min(G[g] for g in kept_g) - max(dropped_g)
+    else:
+        elig = [True] * E
+    sel = _brute_topk(key, K, elig)
+    rest = [key[j] for j in range(E) if elig[j] and j not in sel]
+    topk_gap = min(key[i] for i in sel) - max(rest) if rest else math.inf
+    return topk_gap, group_gap
+
+
+def pin_near_tie_bruteforce(seed=10, trials=240):
+    """near_tie_tokens against enumeration.  Keys are multiples of 2^-12 (sums
+    and differences exact in fp32 and float64) with a threshold of 3 * 2^-12,
+    so gaps of 0 (exact ties), 1 and 2 units are fragile and 3 or more are not;
+    negative keys come from negative biases."""
+    rng = np.random.default_rng(seed)
+    unit = 2.0 ** -12
+    thr = 3 * unit
+    shapes = [(1, 8, 1, 2, 0), (1, 6, 1, 3, 0), (1, 5, 1, 4, 0), (4, 4, 2, 3, 2), (4, 4, 1, 2, 1),
+              (8, 2, 3, 4, 2), (4, 2, 2, 4, 2), (4, 4, 3, 5, 2)]
+    seen = set()
+    for trial in range(trials):
+        n_groups, gsz, keep, K, topn = shapes[trial % len(shapes)]
+        E = n_groups * gsz
+        T = 6
+        s = (rng.integers(0, 24, size=(T, E)) * unit).astype(F32)
+        b = (rng.integers(-12, 4, size=E) * unit).astype(F32)
+        keys = mo.selection_keys(s, b)
+        got = mo.near_tie_tokens(s, b, K, n_groups, keep, topn, gap=thr)
+        for t in range(T):
+            key = [float(v) for v in keys[t]]
+            tg, gg = _brute_gaps(key, K, n_groups, keep, topn)
+            want = tg < thr or gg < thr
+            assert bool(got[t]) == want, (n_groups, gsz, keep, K, topn, key, tg, gg, bool(got[t]))
+            seen.add((want, tg < thr, gg < thr))
+    # both kinds of fragility, and robust tokens, all occurred
+    assert {(True, True, False), (True, False, True), (False, False, False)} <= seen, seen
+
+
+def pin_near_tie_handbuilt():
+    """Hand-built tokens with known gaps.  Threshold 2^-17 with gaps of 2^-18
+    (fragile), exactly 2^-17 (not: the rule is strict) and 2^-16 (not), and the
+    default 1e-5 with gaps of about 0.5e-5 (fragile) and 2e-5 (not)."""
+    def one(key, K, gap, n_groups=1, keep=1, topn=0, b=None):
+        key = np.asarray(key, np.float64)
+        bb = np.zeros(len(key), F32) if b is None else np.asarray(b, F32)
+        s = (key - bb.astype(np.float64)).astype(F32)[None, :]
+        assert np.array_equal(mo.selection_keys(s, bb)[0].astype(np.float64), key), "keys not exact"
+        return bool(mo.near_tie_tokens(s, bb, K, n_groups, keep, topn, gap=gap)[0])
+
+    u = 2.0 ** -17
+    base = [0.75, 0.5, 0.25, 0.125, 0.0625, 0.03125, 0.015625, 0.0078125]
+    for delta, want in ((u / 2, True), (u, False), (2 * u, False)):
+        k = list(base)
+        k[2] = k[1] - delta                      # K = 2: 2nd vs 3rd largest
+        assert one(k, 2, u) == want, delta
+        kn = [v - 1.0 for v in k]                # the same gaps on negative keys (negative bias)
+        assert one(kn, 2, u, b=[-1.0] * 8) == want, delta
+    k = list(base)
+    k[1] = k[0] - u / 2                          # a tie inside the selected set is harmless
+    assert one(k, 2, u) is False
+    k = list(base)
+    k[3] = k[2] - u / 2                          # a tie among the unselected ones is harmless
+    assert one(k, 2, u) is False
+    # default threshold 1e-5 (fp32 keys near 0.5: spacing 6e-8)
+    for delta, want in ((0.5e-5, True), (2e-5, False)):
+        k = [float(F32(v)) for v in (0.9, 0.5, 0.5 - delta, 0.1)]
+        assert one(k, 2, 1e-5) == want, delta
+
+    # 4 groups of 4, keep 2, group score = top-2 sum, K = 2; keys listed group by group
+    def g4(*groups):
+        return [v for grp in groups for v in (list(grp) + [0.0] * (4 - len(grp)))]
+    # group scores 1.0, 0.5, 0.5 - delta, 0.0625: fragile exactly when delta < threshold
+    for delta, want in ((u / 2, True), (u, False), (2 * u, False)):
+        k = g4((0.5, 0.5), (0.25, 0.25), (0.25, 0.25 - delta), (0.0625,))
+        assert one(k, 2, u, 4, 2, 2) == want, delta
+    # the two DROPPED groups tie (0.25 and 0.25), kept groups far apart: harmless;
+    # the best groups are not in index order (scores 1.0, 0.25, 0.25, 0.5)
+    assert one(g4((0.5, 0.5), (0.125, 0.125), (0.125, 0.125), (0.25, 0.25)), 2, u, 4, 2, 2) is False
+    # an expert of a dropped group (score 0.3125 - u/4) nearly ties the K-th
+    # selected key 0.3125, but it is ineligible: harmless
+    k = g4((0.5, 0.125), (0.3125, 0.1875), (0.3125 - u / 4,), (0.0625,))
+    assert one(k, 2, u, 4, 2, 2) is False
+    # the K-th eligible key and the next eligible one (in a kept group) nearly tie
+    k = g4((0.5, 0.375), (0.375 - u / 2, 0.125), (), (0.0625,))
+    assert one(k, 2, u, 4, 2, 2) is True
+
+
+def pin_dense_capacity(seed=11):
+    """Capacity drops in the forward pass: the layer equals the dense
+    all-experts restatement with the gates of dropped pairs set to zero and the
+    surviving gates left as they are.  The kept pairs are found here by walking
+    the tokens in order with a counter per expert (the lowest token indices are
+    admitted first); capacities for T*K = 80 rows over 6 experts are written
+    out by hand: CF 1.0 -> 13, 0.5 -> 6, 0.001 -> 0 (every pair dropped, so
+    y = h + the shared expert)."""
+    rng = np.random.default_rng(seed)
+    T, d, f, fs, E, K, Es = 40, 16, 24, 10, 6, 2, 1
+    h = rng.normal(size=(T, d)).astype(F32)
+    e = (rng.normal(size=(E, d)) * 0.5).astype(F32)
+    e[0] += 1.0                                   # skewed: expert 0 overflows its capacity
+    b = np.zeros(E, F32)
+    W = [rng.normal(size=(E, f, d)), rng.normal(size=(E, f, d)), rng.normal(size=(E, d, f))]
+    sW = [rng.normal(size=(Es, fs, d)), rng.normal(size=(Es, fs, d)), rng.normal(size=(Es, d, fs))]
+    dropped_any = False
+    for cf, C in ((1.0, 13), (0.5, 6), (0.001, 0)):
+        cfg = mo.LayerConfig(T=T, d_model=d, E_r=E, E_s=Es, K=K, capacity_factor=cf)
+        out = mo.layer_forward(cfg, h, e, b, mo.array_weights(*W, *sW))
+        used = [0] * E
+        G = np.zeros((T, E))
+        for t in range(T):
+            for k in range(K):
+                i = int(out["idx"][t, k])
+                if used[i] < C:
+                    G[t, i] = float(out["gates"][t, k])
+                    used[i] += 1
+                else:
+                    dropped_any = True
+        want = _dense_layer(h.astype(np.float64), G, W, sW)
+        assert np.allclose(out["y"], want, rtol=1e-11, atol=1e-11), cf
+        assert out["kept"].tolist() == used, cf
+        if C == 0:
+            assert np.allclose(out["y"], _dense_layer(h.astype(np.float64), np.zeros((T, E)), W, sW),
+                               rtol=1e-12, atol=1e-12)
+    assert dropped_any
+
+
 PINS = [pin_worked_bias_example, pin_bruteforce_topk, pin_bruteforce_grouped, pin_gates_properties,
         pin_counts_and_bias, pin_softmax_closed_form, pin_k_equals_e, pin_dense_reduction,
-        pin_dense_all_experts, pin_capacity, pin_permutation_properties]
+        pin_dense_all_experts, pin_capacity, pin_permutation_properties, pin_near_tie_bruteforce,
+        pin_near_tie_handbuilt, pin_dense_capacity]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -355,6 +504,62 @@ def _mut_counts_kept_only(idx, E_r):      # off-by-one histogram
     return np.concatenate([c, np.zeros(max(0, E_r - len(c)), np.int64)]).astype(np.int64)
 
 
+def _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, *, kth=None, masked=True,
+                      sort_groups=True, groups=True):
+    keys = mo.selection_keys(s32, b32).astype(np.float64)
+    T, E = keys.shape
+    fragile = np.zeros(T, dtype=bool)
+    if groups and n_groups > 1 and group_topn > 0 and topk_groups < n_groups:
+        G = mo.group_scores(mo.selection_keys(s32, b32), n_groups, group_topn).astype(np.float64)
+        if sort_groups:
+            G = np.sort(G, axis=1)[:, ::-1]
+        fragile |= (G[:, topk_groups - 1] - G[:, topk_groups]) < gap
+    elig = mo.eligible_mask(mo.selection_keys(s32, b32), n_groups, topk_groups, group_topn)
+    srt = -np.sort(-(np.where(elig, keys, -np.inf) if masked else keys), axis=1)
+    k = K if kth is None else kth
+    if 1 <= k < E:
+        nxt = srt[:, k]
+        fragile |= np.isfinite(nxt) & ((srt[:, k - 1] - nxt) < gap)
+    return fragile
+
+
+def _mut_near_tie_gap_after_k(s32, b32, K, n_groups=1, topk_groups=1, group_topn=0, gap=1e-5):
+    return _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, kth=K + 1)
+
+
+def _mut_near_tie_gap_inside(s32, b32, K, n_groups=1, topk_groups=1, group_topn=0, gap=1e-5):
+    return _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, kth=K - 1)
+
+
+def _mut_near_tie_unmasked(s32, b32, K, n_groups=1, topk_groups=1, group_topn=0, gap=1e-5):
+    return _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, masked=False)
+
+
+def _mut_near_tie_groups_unsorted(s32, b32, K, n_groups=1, topk_groups=1, group_topn=0, gap=1e-5):
+    return _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, sort_groups=False)
+
+
+def _mut_near_tie_no_group_gap(s32, b32, K, n_groups=1, topk_groups=1, group_topn=0, gap=1e-5):
+    return _near_tie_variant(s32, b32, K, n_groups, topk_groups, group_topn, gap, groups=False)
+
+
+def _mut_layer_output_ignores_drops(cfg, h, idx, gates, disp, weights, tokens=None):
+    full = mo.Dispatch(disp.counts, disp.counts, disp.offsets, disp.perm_tok, disp.perm_slot,
+                       np.zeros_like(disp.row_of))
+    return _orig_layer_output(cfg, h, idx, gates, full, weights, tokens)
+
+
+def _mut_layer_output_renormalises(cfg, h, idx, gates, disp, weights, tokens=None):
+    kept = disp.row_of >= 0
+    g = np.where(kept, gates, 0).astype(np.float64)
+    ssum = g.sum(1, keepdims=True)
+    g = np.where(ssum > 0, g / np.where(ssum > 0, ssum, 1), 0).astype(F32)
+    return _orig_layer_output(cfg, h, idx, g, disp, weights, tokens)
+
+
+_orig_layer_output = mo.layer_output
+
+
 MUTATIONS = [
     ("bias_update", _mut_bias_sign),
     ("bias_update", _mut_sign_zero_up),
@@ -366,6 +571,13 @@ MUTATIONS = [
     ("group_scores", _mut_group_sum_top1),
     ("selection_keys", _mut_selection_ignores_bias),
     ("load_counts", _mut_counts_kept_only),
+    ("near_tie_tokens", _mut_near_tie_gap_after_k),
+    ("near_tie_tokens", _mut_near_tie_gap_inside),
+    ("near_tie_tokens", _mut_near_tie_unmasked),
+    ("near_tie_tokens", _mut_near_tie_groups_unsorted),
+    ("near_tie_tokens", _mut_near_tie_no_group_gap),
+    ("layer_output", _mut_layer_output_ignores_drops),
+    ("layer_output", _mut_layer_output_renormalises),
 ]
 
 
