@@ -12,6 +12,17 @@ weights (22.6 GB) are far larger than L2, so no flush is needed.  N > 1 runs N
 independent replicas (one process per GPU, no collective in the data path):
 weak scaling, timed as the max over ranks.
 
+At N = 1 the line also carries "workloads": one sub-record per other
+configuration (decode-sized DeepSeek-V3, Mixtral-style, fine-grained dropless
+and with capacity factor 1.25, the fp32 toy), each timed alone on the same GPU
+with its own layer roofline, kernel rooflines and clocks (--workloads none
+skips them).
+
+Roofline bytes follow the definition: touched expert weights, shared weights,
+centroids, h in and y out for the layer; for the gate/up GEMM (the dominant
+kernel) its touched weights and h read once.  Permuted copies and
+intermediates are implementation costs and are reported separately.
+
 --impl reference times the CPU oracle (oracle/) on the host cores on a bounded
 sample of the same workload (rank 0 only).
 """
@@ -71,38 +82,55 @@ def layer_work(w, kept: np.ndarray):
     return flops, nbytes
 
 
+def _weight_bytes(w, rows: int, cols: int) -> int:
+    """Bytes of one expert weight matrix [rows, cols]: bf16 (2 B), fp32 (4 B), or
+    e4m3 codes (1 B) plus one fp32 scale per row."""
+    if w.dtype == "bf16_e4m3":
+        return rows * cols + 4 * rows
+    return rows * cols * (4 if w.dtype == "f32" else 2)
+
+
 def gateup_work(w, kept: np.ndarray):
-    """(flops, bytes) of one launch of the gate/up grouped GEMM: touched gate+up
-    weights, one read of the permuted rows (and of h for the shared experts),
-    one write of the SwiGLU products."""
+    """(flops, bytes) of one launch of the gate/up grouped GEMM by the roofline
+    definition: the gate and up weights of every touched routed expert and of
+    the shared experts, and the token rows h read once.  The permuted copy of
+    the rows and the SwiGLU products are implementation costs, not counted."""
     n_rows = int(kept.sum())
     touched = int((kept > 0).sum())
     d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
-    rows_s = w.E_s * w.T
-    flops = 4 * d * (f * n_rows + fs * rows_s)
-    if w.dtype == "bf16_e4m3":
-        # e4m3 weights and rows (+ fp32 row scales), bf16 SwiGLU products out
-        x_rows = n_rows + min(rows_s, w.T)
-        nbytes = (touched * 2 * (d * f + 4 * f) + w.E_s * 2 * (d * fs + 4 * fs) + x_rows * (d + 4)
-                  + 2 * (n_rows * f + rows_s * fs))
-    else:
-        nbytes = 2 * (touched * 2 * d * f + w.E_s * 2 * d * fs + (n_rows + min(rows_s, w.T)) * d
-                      + n_rows * f + rows_s * fs)
+    flops = 4 * d * (f * n_rows + fs * w.E_s * w.T)
+    es = 4 if w.dtype == "f32" else 2
+    nbytes = 2 * touched * _weight_bytes(w, f, d) + 2 * w.E_s * _weight_bytes(w, fs, d) + w.T * d * es
     return flops, nbytes
 
 
 def down_work(w, kept: np.ndarray):
+    """(flops, bytes) of one launch of the down grouped GEMM by the roofline
+    definition: the W_down of every touched routed expert and of the shared
+    experts, and the layer output written once."""
+    n_rows = int(kept.sum())
+    touched = int((kept > 0).sum())
+    d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
+    flops = 2 * d * (f * n_rows + fs * w.E_s * w.T)
+    es = 4 if w.dtype == "f32" else 2
+    nbytes = touched * _weight_bytes(w, d, f) + w.E_s * _weight_bytes(w, d, fs) + w.T * d * es
+    return flops, nbytes
+
+
+def gateup_impl_bytes(w, kept: np.ndarray) -> int:
+    """Bytes the gate/up launch moves as implemented: the weights, one read of
+    every permuted row (and of h for the shared experts) and one write of the
+    SwiGLU products (the basis of the DRAM-traffic ratio in profiles/)."""
     n_rows = int(kept.sum())
     touched = int((kept > 0).sum())
     d, f, fs = w.d_model, w.d_ffn, w.d_ffn_shared
     rows_s = w.E_s * w.T
-    flops = 2 * d * (f * n_rows + fs * rows_s)
     if w.dtype == "bf16_e4m3":
-        nbytes = (touched * (d * f + 4 * d) + w.E_s * (d * fs + 4 * d) + n_rows * (f + 4)
-                  + rows_s * (fs + 4) + 2 * (n_rows + rows_s) * d)
-    else:
-        nbytes = 2 * (touched * d * f + w.E_s * d * fs + n_rows * f + rows_s * fs + (n_rows + rows_s) * d)
-    return flops, nbytes
+        x_rows = n_rows + min(rows_s, w.T)
+        return (touched * 2 * (d * f + 4 * f) + w.E_s * 2 * (d * fs + 4 * fs) + x_rows * (d + 4)
+                + 2 * (n_rows * f + rows_s * fs))
+    return 2 * (touched * 2 * d * f + w.E_s * 2 * d * fs + (n_rows + min(rows_s, w.T)) * d
+                + n_rows * f + rows_s * fs)
 
 
 # ---------------------------------------------------------------------------
@@ -147,7 +175,7 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, window=None):
         import datetime
         rows = []
         for ln in self.lines:
@@ -159,8 +187,9 @@ class ClockSampler:
                 rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
             except ValueError:
                 continue
-        if self.window:
-            lo, hi = self.window
+        window = window or self.window
+        if window:
+            lo, hi = window
             inside = [r for r in rows if lo <= r[0] <= hi]
         else:
             inside = rows
@@ -365,7 +394,7 @@ def run_train(args, w, rank, world, local_rank):
     if rank != 0:
         return
     peaks, peak_kind = load_peaks()
-    hbm, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops_sustained"])
+    hbm, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
     tw = [train_work(w, k) for k in kept_h]
     b_flops, b_bytes = float(np.mean([x[0] for x in tw])), float(np.mean([x[1] for x in tw]))
     bwd_s = float(np.mean(bwd)) / 1000
@@ -388,7 +417,7 @@ def run_train(args, w, rank, world, local_rank):
                               "flops": b_flops, "bytes": b_bytes,
                               "bound": "hbm" if b_bytes / (hbm * 1e9) >= b_flops / (bf16_peak * 1e12) else "tensor",
                               "achieved_gbs": b_bytes / bwd_s / 1e9, "achieved_tflops": b_flops / bwd_s / 1e12,
-                              "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s sustained",
+                              "peaks": f"{peak_kind}: {hbm} GB/s, {bf16_peak} TFLOP/s burst",
                               "write_aware": {"t_roof_ms": 1000 * t_roof_w, "frac": 1000 * t_roof_w / float(np.mean(bwd)),
                                               "writes": b_writes, "write_gbs": write_gbs,
                                               "note": "writes at the write-only bandwidth measured live "
@@ -436,7 +465,7 @@ def run_reference(args, w, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000 * total / len(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w),
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                              "kind": "oracle",
                              "sample": f"each step: {per_step} seeded tokens of the batch, full layer "
@@ -485,20 +514,13 @@ def job_throughput(world: int, tokens_per_step: int, steps: int, max_ms: float) 
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, w, rank, world, local_rank):
+def make_inputs(w, dev, stream, rank, n_steps, moe, native):
+    """Device-resident inputs of a workload: weights (e4m3 blobs for the
+    e4m3-weight layers), centroids, bias and one fresh token batch per step."""
     import torch
-    import torch.distributed as dist
-    import sparse_mixture_experts_selection_b200 as moe
-    from moe_inputs import native
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream()
     bf16 = w.dtype != "f32"                 # bf16 activations (bf16 and e4m3-weight layers)
     e4m3 = w.dtype == "bf16_e4m3"
     dt = torch.bfloat16 if bf16 else torch.float32
-
-    # ---- inputs resident in HBM ----
     W = {}
     for k in ("gate", "up", "down", "sgate", "sup", "sdown"):
         tid, n, rows, cols, sigma = mi.weight_spec(w, k)
@@ -517,65 +539,196 @@ def run_ours(args, w, rank, world, local_rank):
         W[k] = t
     e = torch.from_numpy(mi.gen_centroids(w)).to(dev)
     b = torch.from_numpy(mi.gen_bias(w)).to(dev)
-    n_steps = args.warmup + args.steps
     H = []
     for i in range(n_steps):
         t = torch.empty((w.T, w.d_model), dtype=dt, device=dev)
         native.fill_device(t.data_ptr(), t.numel(), bf16, w.seed, h_stream_id(rank, i), 0, 1.0,
                            stream=stream.cuda_stream)
         H.append(t)
-    cfg = moe.config_for(w)
-    ws = moe.alloc_workspace(moe.moe_workspace_size(cfg), dev)
-    y = torch.empty((w.T, w.d_model), dtype=dt, device=dev)
-    kept = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
-    counts = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
-    max_vio = torch.zeros(n_steps, dtype=torch.float32, device=dev)
-    update = w.gamma > 0
+    return {"W": W, "e": e, "b": b, "H": H, "dt": dt}
 
-    def step(i, hh=None, yy=None):
-        moe.moe_layer_forward(cfg, H[i] if hh is None else hh, e, b, W["gate"], W["up"], W["down"],
-                              W["sgate"], W["sup"], W["sdown"], y if yy is None else yy, ws,
-                              counts_out=counts[i],
-                              kept_out=kept[i], update_bias=update, gamma=w.gamma,
-                              max_vio_out=max_vio[i:i + 1])
 
+class LayerRun:
+    """moe_layer_forward (with the bias step when the workload has one) over
+    the workload's fresh batches, with phase events and per-step loads."""
+
+    def __init__(self, w, inp, dev, moe, n_steps):
+        import torch
+        self.w, self.inp, self.moe = w, inp, moe
+        self.cfg = moe.config_for(w)
+        self.ws = moe.alloc_workspace(moe.moe_workspace_size(self.cfg), dev)
+        self.y = torch.empty((w.T, w.d_model), dtype=inp["dt"], device=dev)
+        self.kept = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
+        self.counts = torch.zeros((n_steps, w.E_r), dtype=torch.int32, device=dev)
+        self.max_vio = torch.zeros(n_steps, dtype=torch.float32, device=dev)
+
+    def step(self, i, hh=None, yy=None):
+        W, inp, w = self.inp["W"], self.inp, self.w
+        self.moe.moe_layer_forward(self.cfg, inp["H"][i] if hh is None else hh, inp["e"], inp["b"], W["gate"],
+                                   W["up"], W["down"], W["sgate"], W["sup"], W["sdown"],
+                                   self.y if yy is None else yy, self.ws, counts_out=self.counts[i],
+                                   kept_out=self.kept[i], update_bias=w.gamma > 0, gamma=w.gamma,
+                                   max_vio_out=self.max_vio[i:i + 1])
+
+    def timed(self, first, steps, world, dev, clocks=None):
+        """Time steps first .. first+steps-1 (CUDA events on the launch stream,
+        barrier + synchronize on both sides, max over ranks); returns
+        (elapsed_ms, phase_ms [steps, phases], clock summary)."""
+        import torch
+        import torch.distributed as dist
+        moe = self.moe
+        n_ph = len(moe.PHASES) + 1
+        ph_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ph)] for _ in range(steps)]
+        for evs in ph_events:
+            for ev in evs:
+                ev.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        wall0 = time.time()
+        t_start.record()
+        for j in range(steps):
+            moe.moe_set_phase_events(ph_events[j])
+            self.step(first + j)
+        t_end.record()
+        torch.cuda.synchronize()
+        wall1 = time.time()
+        moe.moe_set_phase_events([])
+        if world > 1:
+            dist.barrier()
+        elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+        err = moe.moe_get_device_error(self.ws)
+        if err:
+            raise RuntimeError(f"device error word {err} after the timed region")
+        phase_ms = np.array([[evs[i].elapsed_time(evs[i + 1]) for i in range(n_ph - 1)] for evs in ph_events])
+        clk = clocks.summary((wall0, wall1)) if clocks else None
+        return elapsed_ms, phase_ms, clk
+
+
+def kernel_records(w, kept_h, phase_ms, ms_per_step, moe):
+    """Roofline records of the step and of its two grouped GEMMs (the gate/up
+    GEMM is the dominant kernel), by the roofline definition's bytes and
+    FLOPs, against the measured peaks (burst GEMM figure: the timed regions
+    last well under a second)."""
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    e4m3 = w.dtype == "bf16_e4m3"
+    # e4m3 tensor-core peak: the measured bf16 figure x the nominal fp8/bf16 ratio (4.5 / 2.25)
+    mma_peak = float(peaks["bf16_tflops"]) * (2.0 if e4m3 else 1.0)
+    peak_note = f"{peak_kind}: {hbm} GB/s, {mma_peak} TFLOP/s burst" + (" (e4m3: bf16 x 2, nominal ratio)" if e4m3 else "")
+    gu_s = float(np.mean(phase_ms[:, moe.PHASES.index("ffn_gate_up")])) / 1000.0
+    dn_s = float(np.mean(phase_ms[:, moe.PHASES.index("ffn_down")])) / 1000.0
+    mean = lambda f: tuple(float(np.mean([f(w, k)[i] for k in kept_h])) for i in range(2))
+    gu_flops, gu_bytes = mean(gateup_work)
+    dn_flops, dn_bytes = mean(down_work)
+    l_flops, l_bytes = mean(layer_work)
+    gu_impl = float(np.mean([gateup_impl_bytes(w, k) for k in kept_h]))
+    t_roof = max(l_flops / (mma_peak * 1e12), l_bytes / (hbm * 1e9))
+    gu = {"bound": "hbm" if gu_bytes / (hbm * 1e9) >= gu_flops / (mma_peak * 1e12) else "tensor",
+          "achieved_gbs": gu_bytes / gu_s / 1e9, "frac_hbm": gu_bytes / gu_s / 1e9 / hbm,
+          "achieved_tflops": gu_flops / gu_s / 1e12, "frac_tensor": gu_flops / gu_s / 1e12 / mma_peak,
+          "ms": 1000 * gu_s, "bytes": gu_bytes, "flops": gu_flops,
+          "impl_bytes": gu_impl, "kernel_traffic_frac": gu_impl / gu_s / 1e9 / hbm}
+    dn = {"achieved_gbs": dn_bytes / dn_s / 1e9, "frac_hbm": dn_bytes / dn_s / 1e9 / hbm,
+          "achieved_tflops": dn_flops / dn_s / 1e12, "frac_tensor": dn_flops / dn_s / 1e12 / mma_peak,
+          "ms": 1000 * dn_s, "bytes": dn_bytes, "flops": dn_flops}
+    layer = {"t_roof_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms_per_step, "flops": l_flops, "bytes": l_bytes,
+             "bound": "hbm" if l_bytes / (hbm * 1e9) >= l_flops / (mma_peak * 1e12) else "tensor",
+             "frac_hbm": l_bytes / (hbm * 1e9) * 1000 / ms_per_step,
+             "frac_tensor": l_flops / (mma_peak * 1e12) * 1000 / ms_per_step, "peaks": peak_note}
+    return gu, dn, layer, hbm, mma_peak, peak_kind
+
+
+def launches_per_step(w) -> int:
+    """Our kernels per layer step: [centroid split + router GEMM | CUDA-core
+    logits], select, scan, scatter, gather (e4m3: quantize h + gather), group
+    tables, gate/up GEMM, down GEMM, combine, bias step; e4m3 adds the
+    quantization of A (and of the shared A when there are shared experts)."""
+    bf16 = w.dtype != "f32"
+    e4m3 = w.dtype == "bf16_e4m3"
+    return (11 if bf16 else 10) + ((1 + 2 * (w.E_s > 0)) if e4m3 else 0)
+
+
+def measure_extra(name, args, rank, world, dev, stream, moe, native, clocks):
+    """One sub-record: a workload timed alone on this GPU (at least ~200 ms of
+    timed steps so that the clock samples cover it)."""
+    import torch
+    w = mi.WORKLOADS[name]
+    warm = args.warmup
+    probe = make_inputs(w, dev, stream, rank, warm, moe, native)
+    run = LayerRun(w, probe, dev, moe, warm)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(warm):
+        run.step(i)
+    b_.record()
+    torch.cuda.synchronize()
+    est_ms = a.elapsed_time(b_) / warm
+    steps = int(min(4000, max(args.steps, math.ceil(200.0 / max(est_ms, 1e-3)))))
+    del run
+    # fresh batches for warm-up + timed steps; the weights of the probe are reused
+    H = []
+    for i in range(warm + steps):
+        t = torch.empty((w.T, w.d_model), dtype=probe["dt"], device=dev)
+        native.fill_device(t.data_ptr(), t.numel(), w.dtype != "f32", w.seed, h_stream_id(rank, i), 0, 1.0,
+                           stream=stream.cuda_stream)
+        H.append(t)
+    inp = dict(probe, H=H, b=torch.from_numpy(mi.gen_bias(w)).to(dev))
+    run = LayerRun(w, inp, dev, moe, warm + steps)
+    for i in range(warm):
+        run.step(i)
+    torch.cuda.synchronize()
+    elapsed_ms, phase_ms, clk = run.timed(warm, steps, world, dev, clocks)
+    ms = elapsed_ms / steps
+    kept_h = run.kept.cpu().numpy()[warm:]
+    counts_h = run.counts.cpu().numpy()[warm:]
+    gu, dn, layer, _, _, _ = kernel_records(w, kept_h, phase_ms, ms, moe)
+    rec = {"value": job_throughput(world, w.T, steps, elapsed_ms), "unit": "tokens/s", "ms_per_step": ms,
+           "steps": steps, "warmup": warm, "dtype": {"bf16": "bf16", "bf16_e4m3": "e4m3"}.get(w.dtype, "f32"),
+           "config": workload_config(w), "layer_roofline": layer, "gate_up_gemm": gu, "down_gemm": dn,
+           "phases_ms": {p: float(np.mean(phase_ms[:, i])) for i, p in enumerate(moe.PHASES)},
+           "rows_per_step": float(np.mean(kept_h.sum(1))), "touched_experts": float(np.mean((kept_h > 0).sum(1))),
+           "dropped_pairs_per_step": float(np.mean(counts_h.sum(1) - kept_h.sum(1))),
+           "clocks": clk, "gpu_launches": launches_per_step(w) * steps}
+    if w.gamma > 0:
+        vio = run.max_vio.cpu().numpy()[warm:]
+        rec["max_vio_first_last"] = [round(float(vio[0]), 4), round(float(vio[-1]), 4)]
+    del run, inp, probe, H
+    torch.cuda.empty_cache()
+    return rec
+
+
+EXTRA_WORKLOADS = ["deepseek_v3_decode", "mixtral_8x14336", "finegrained_64x1408", "finegrained_64x1408_cf1.25",
+                   "toy_fp32"]
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_mixture_experts_selection_b200 as moe
+    from moe_inputs import native
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    bf16 = w.dtype != "f32"
+    e4m3 = w.dtype == "bf16_e4m3"
+    dt = torch.bfloat16 if bf16 else torch.float32
     clocks = ClockSampler(torch.cuda.current_device())
+
+    # ---- inputs resident in HBM ----
+    n_steps = args.warmup + args.steps
+    inp = make_inputs(w, dev, stream, rank, n_steps, moe, native)
+    run = LayerRun(w, inp, dev, moe, n_steps)
     for i in range(args.warmup):
-        step(i)
+        run.step(i)
     torch.cuda.synchronize()
-    b_after_warmup = b.clone()
-
-    # phase events per timed step
-    n_ph = len(moe.PHASES) + 1
-    ph_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ph)] for _ in range(args.steps)]
-    for evs in ph_events:
-        for ev in evs:
-            ev.record()
-    torch.cuda.synchronize()
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    wall0 = time.time()
-    t_start.record()
-    for j in range(args.steps):
-        moe.moe_set_phase_events(ph_events[j])
-        step(args.warmup + j)
-    t_end.record()
-    torch.cuda.synchronize()
-    clocks.mark(wall0, time.time())
-    moe.moe_set_phase_events([])
-    if world > 1:
-        dist.barrier()
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
-    err = moe.moe_get_device_error(ws)
-    if err:
-        raise RuntimeError(f"device error word {err} after the timed region")
-
-    phase_ms = np.array([[evs[i].elapsed_time(evs[i + 1]) for i in range(n_ph - 1)] for evs in ph_events])
-    kept_h = kept.cpu().numpy()[args.warmup:]
-    vio_h = max_vio.cpu().numpy()
+    b_after_warmup = inp["b"].clone()
+    elapsed_ms, phase_ms, clk = run.timed(args.warmup, args.steps, world, dev, clocks)
+    kept_h = run.kept.cpu().numpy()[args.warmup:]
+    vio_h = run.max_vio.cpu().numpy()
     value = job_throughput(world, w.T, args.steps, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
 
@@ -586,11 +739,12 @@ def run_ours(args, w, rank, world, local_rank):
         # every step.  Copies run on a second stream, double-buffered, so the
         # H2D of step j+1 and the D2H of step j overlap the compute of the
         # neighbouring steps; the timed region spans the first H2D to the last D2H.
+        H = inp["H"]
         pin_h = [H[i].cpu().pin_memory() for i in range(args.warmup, n_steps)]
         y_host = [torch.empty((w.T, w.d_model), dtype=dt).pin_memory() for _ in range(2)]
         h_dev = [torch.empty_like(H[0]) for _ in range(2)]
-        y_dev = [y, torch.empty_like(y)]
-        b.copy_(b_after_warmup)
+        y_dev = [run.y, torch.empty_like(run.y)]
+        inp["b"].copy_(b_after_warmup)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -610,7 +764,7 @@ def run_ours(args, w, rank, world, local_rank):
             main.wait_event(h_ready[j])
             if j >= 2:
                 main.wait_event(y_read[j - 2])          # y_dev[buf] has been read back
-            step(args.warmup + j, h_dev[buf], y_dev[buf])
+            run.step(args.warmup + j, h_dev[buf], y_dev[buf])
             done[j].record(main)
             with torch.cuda.stream(cs):
                 if j + 1 < args.steps:
@@ -629,25 +783,11 @@ def run_ours(args, w, rank, world, local_rank):
         e2e = {"value": job_throughput(world, w.T, args.steps, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": w.T * w.d_model * es, "d2h_bytes_per_step": w.T * w.d_model * es,
                "copies": "pinned host, second stream, double-buffered"}
+        del pin_h, y_host, h_dev, y_dev
 
-    clocks.stop()
-    if rank != 0:
-        return
-
-    peaks, peak_kind = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    bf16_peak = float(peaks["bf16_tflops_sustained"])
-    # dominant kernel: the gate/up grouped GEMM
-    gu_ms = phase_ms[:, moe.PHASES.index("ffn_gate_up")]
-    dn_ms = phase_ms[:, moe.PHASES.index("ffn_down")]
-    gu = [gateup_work(w, k) for k in kept_h]
-    dn = [down_work(w, k) for k in kept_h]
-    gu_bytes = float(np.mean([x[1] for x in gu]))
-    gu_flops = float(np.mean([x[0] for x in gu]))
-    gu_s = float(np.mean(gu_ms)) / 1000.0
-    achieved = gu_bytes / gu_s / 1e9
-    # DRAM traffic per launch: the ncu capture's traffic/algorithmic ratio
-    # (profiles/traffic.json) scaled to this launch's algorithmic bytes
+    gu, dn, layer, hbm, mma_peak, peak_kind = kernel_records(w, kept_h, phase_ms, ms_per_step, moe)
+    # DRAM traffic per launch: the ncu capture's DRAM bytes over its implementation
+    # bytes (profiles/traffic.json), scaled to this launch's implementation bytes
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -658,42 +798,41 @@ def run_ours(args, w, rank, world, local_rank):
         # counters taken on another version of the kernel say nothing about this one
         same = os.path.isfile(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == doc.get("source_sha256")
         if rec and same and w.dtype == "bf16":       # counters of the bf16 kernel
-            traffic = rec["ratio"] * gu_bytes
-    layer = [layer_work(w, k) for k in kept_h]
-    l_flops = float(np.mean([x[0] for x in layer]))
-    l_bytes = float(np.mean([x[1] for x in layer]))
-    # e4m3 tensor-core peak: the measured bf16 figure x the nominal fp8/bf16 ratio (4.5 / 2.25)
-    mma_peak = bf16_peak * (2.0 if e4m3 else 1.0)
-    t_roof = max(l_flops / (mma_peak * 1e12), l_bytes / (hbm * 1e9))
+            traffic = rec["ratio"] * gu["impl_bytes"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if e4m3 else ("bf16" if bf16 else "f32"),
         "data": "synthetic", "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic, "kernel": "ffn_gate_up (tcgen05 grouped GEMM)",
-                     "peak_source": f"{peak_kind} hbm_gbs",
-                     "tensor_tflops": gu_flops / gu_s / 1e12,
-                     "tensor_frac_sustained": gu_flops / gu_s / 1e12 / mma_peak},
-        "layer_roofline": {"t_roof_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms_per_step,
-                           "flops": l_flops, "bytes": l_bytes,
-                           "bound": "hbm" if l_bytes / (hbm * 1e9) >= l_flops / (mma_peak * 1e12) else "tensor",
-                           "peaks": f"{peak_kind}: {hbm} GB/s, {mma_peak} TFLOP/s sustained"
-                                    + (" (e4m3: bf16 x 2, nominal ratio)" if e4m3 else "")},
+        "roofline": {"bound": "hbm", "achieved": gu["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                     "frac": gu["frac_hbm"], "traffic": traffic,
+                     "kernel": "ffn_gate_up (tcgen05 grouped GEMM)",
+                     "bytes_per_launch": gu["bytes"],
+                     "bytes_def": "touched routed gate+up weights + shared gate+up weights + h read once",
+                     "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})",
+                     "kernel_traffic_frac": gu["kernel_traffic_frac"],
+                     "kernel_traffic_note": "implementation bytes (adds the permuted-row read and the "
+                                            "SwiGLU-product write) over the same time",
+                     "tensor_tflops": gu["achieved_tflops"], "tensor_frac_burst": gu["frac_tensor"]},
+        "layer_roofline": layer,
         "phases_ms": {p: float(np.mean(phase_ms[:, i])) for i, p in enumerate(moe.PHASES)},
-        "down_gemm": {"achieved_gbs": float(np.mean([x[1] for x in dn])) / (float(np.mean(dn_ms)) / 1000) / 1e9},
+        "down_gemm": dn,
         "rows_per_step": float(np.mean(kept_h.sum(1))),
         "touched_experts": float(np.mean((kept_h > 0).sum(1))),
         "max_vio": [round(float(v), 4) for v in vio_h[args.warmup:]],
         "e2e": e2e,
-        "clocks": clocks.summary(),
-        # our kernels per step: [centroid split + router GEMM | CUDA-core logits], select,
-        # scan, scatter, gather, group tables, gate/up GEMM, down GEMM, combine, bias step
-        # per step: split, router GEMM, select, scan, scatter, gather (e4m3: gather +
-        # quantize), groups, gate/up, down, combine, bias; e4m3 adds the quantization
-        # of A, and of h and the shared A when there are shared experts
-        "gpu_launches": ((11 if bf16 else 10) + ((1 + 2 * (w.E_s > 0)) if e4m3 else 0)) * args.steps,
+        "clocks": clk,
+        "gpu_launches": launches_per_step(w) * args.steps,
     }
+    del run, inp
+    torch.cuda.empty_cache()
+    if world == 1 and args.workloads != "none":
+        names = EXTRA_WORKLOADS if args.workloads == "all" else [n for n in args.workloads.split(",") if n]
+        line["workloads"] = {n: measure_extra(n, args, rank, world, dev, stream, moe, native, clocks)
+                             for n in names if n != w.name}
+    clocks.stop()
+    if rank != 0:
+        return
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
     print(json.dumps(line), flush=True)
@@ -710,6 +849,9 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workloads", default="all",
+                    help="sub-records of the N=1 line: 'all' (the other configurations), 'none', or a "
+                         "comma-separated list of workload names")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (forward with train = 1 + moe_layer_backward)")
     ap.add_argument("--tokens", type=int, default=0,
