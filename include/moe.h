@@ -278,6 +278,36 @@ moe_status moe_gather_rows(const void* src, int64_t n_src, int32_t row_bytes, co
                            int64_t n_rows, void* dst, void* stream);
 
 /*
+ * Exchange plan of an expert-parallel layer ("Sparse Mixture-of-Experts ...",
+ * section 3: dispatch to the experts' ranks, grouped GEMM over the local
+ * experts, combine; "Mixture-of-Experts: Expert Parallelism, All-to-All
+ * Routing, ...", all-to-all routing).  The E_r routed experts are split over
+ * `world` ranks, rank r owning experts r*E_loc .. (r+1)*E_loc - 1
+ * (E_loc = E_r / world); every rank has permuted its own kept rows with
+ * moe_permute, so its rows for rank r are one contiguous range.
+ *   offsets_all [world, E_r + 1] int32: every rank's moe_permute offsets
+ *                (all-gathered), DEVICE.
+ *   splits      [2 * world] int32 out: rows this rank sends to each rank, then
+ *                rows it receives from each rank (the all-to-all split sizes).
+ *   local_offsets [E_loc + 1] int32 out: rows of each local expert after the
+ *                regroup.
+ *   regroup     [max_recv] int32 out: regrouped row j comes from received
+ *                row regroup[j] -- received rows arrive source by source, the
+ *                regroup orders them expert by expert, sources ascending, each
+ *                source's rows in their order.
+ *   inverse     [max_recv] int32 out: inverse[regroup[j]] = j.
+ *   dev_error   optional int32 DEVICE word: set to MOE_DEVERR_INDEX when the
+ *                offsets decrease or more than max_recv rows would arrive (the
+ *                maps are then not written; splits still are).
+ * 1 <= world <= 64, 0 <= rank < world, E_r <= 1024 and divisible by world.
+ * Enqueues one kernel; the caller copies `splits` to the host if its
+ * all-to-all needs them there.
+ */
+moe_status moe_ep_plan(const int32_t* offsets_all, int32_t world, int32_t rank, int32_t E_r,
+                       int32_t max_recv, int32_t* splits, int32_t* local_offsets, int32_t* regroup,
+                       int32_t* inverse, int32_t* dev_error, void* stream);
+
+/*
  * Backward of moe_layer_forward (train = 1): gradients of a loss L, given
  * dy = dL/dy [T, d] (bf16), with respect to h, the centroids e and every
  * expert weight, for the routing the forward chose.  The derivative of the
@@ -343,9 +373,10 @@ moe_status moe_router_stats(const moe_config* cfg, const float* s, const float* 
  * Scratch: a fixed 2 MiB + 64 KiB array in the library's own device memory,
  * held on every GPU that loads the library until exit.  Shapes needing more
  * (2 * ceil(T/256) * E_r + E_r + 64 int32 words) return MOE_ERR_UNSUPPORTED
- * before anything is enqueued.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and must therefore come before
- * any stream capture.  All calls share the array and it keeps the last call's
+ * before anything is enqueued.  The first call in each CUDA context (once per
+ * device for the primary context; again after cudaDeviceReset rebuilds it)
+ * looks up the array's device address (cudaGetSymbolAddress) and must
+ * therefore come before any stream capture.  All calls share the array and it keeps the last call's
  * contents (the call clears what must start at zero): calls whose work
  * overlaps on the GPU, e.g. on two streams, race and must be serialised by the
  * caller.  No cudaMalloc/cudaFree or allocating library routine is called.

@@ -23,7 +23,7 @@ __all__ = [
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
     "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
     "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3", "moe_layer_backward", "moe_gather_rows",
-    "moe_set_phase_events", "moe_selftest_bounded_wait",
+    "moe_set_phase_events", "moe_selftest_bounded_wait", "moe_ep_plan",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
 
@@ -75,6 +75,7 @@ SIGNATURES = {
     "moe_layer_backward": (ctypes.c_int, [_P] * 20 + [_P, ctypes.c_size_t, _P]),
     "moe_quantize_rows": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _I32, _P, _P]),
     "moe_gather_rows": (ctypes.c_int, [_P, ctypes.c_int64, _I32, _P, ctypes.c_int64, _P, _P]),
+    "moe_ep_plan": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "moe_router_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "moe_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32)]),
@@ -220,6 +221,13 @@ def moe_permute_noalloc(cfg, idx, gates, h, offsets, perm_tok, row_of, kept, row
     _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _ptr(idx), _ptr(gates), _ptr(h), _ptr(offsets),
                                      _ptr(perm_tok), _ptr(row_of), _ptr(kept), _ptr(row_gate),
                                      _ptr(x_perm), _ptr(dev_error), _stream(stream)))
+
+
+def moe_ep_plan(offsets_all, world, rank, E_r, max_recv, splits, local_offsets, regroup, inverse,
+                dev_error=None, stream=None):
+    """Exchange plan of an expert-parallel layer on the device (see include/moe.h)."""
+    _check(lib().moe_ep_plan(_ptr(offsets_all), world, rank, E_r, max_recv, _ptr(splits), _ptr(local_offsets),
+                             _ptr(regroup), _ptr(inverse), _ptr(dev_error), _stream(stream)))
 
 
 def moe_expert_ffn(cfg, n_experts, d_ffn, max_rows, offsets, x, w_gate, w_up, w_down, row_scale,

@@ -12,13 +12,18 @@
 //
 // The scratch is one file-scope __device__ array, reserved on every GPU that
 // loads the library until the process exits.  Its device address is looked
-// up once per device (cudaGetSymbolAddress, with that device current) on the
-// first call made on that device, so that first call must come before any
-// stream capture.  Every call on a device shares the array and it keeps the
-// last call's contents: the histogram is cleared at the start of each call,
-// and calls whose work overlaps on the GPU (concurrent streams) race on it.
+// up (cudaGetSymbolAddress, with that device current) on the first call made
+// in each CUDA context -- once per device for the usual primary context, and
+// again after a context has been torn down and rebuilt (cudaDeviceReset),
+// when the array may sit elsewhere -- so the first call in a context must come
+// before any stream capture.  Every call on a device shares the array and it
+// keeps the last call's contents: the histogram is cleared at the start of
+// each call, and calls whose work overlaps on the GPU (concurrent streams)
+// race on it.
 #include <cmath>
 #include <mutex>
+
+#include <cuda.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -32,23 +37,65 @@ static __device__ __align__(256) int g_permute_scratch[kScratchInts];
 
 namespace {
 
-std::mutex g_mu;
-int* g_scratch_ptr[64] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (looked up once).
+// Unique id of the calling thread's current CUDA context (false when no
+// context is current yet or the driver cannot say).  Ids are never reused
+// within a process, unlike context handles.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    looked_up = true;
+  }
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+struct ScratchSlot {
+  int* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+
+std::mutex g_mu;
+ScratchSlot g_slot[64];
+
+// Device address of the scratch array in the current context: looked up on
+// the first call in each context, then served from the per-device cache as
+// long as the same context is current.
 cudaError_t scratch_address(int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_slot[dev];
+  unsigned long long id = 0;
+  const bool known = current_context_id(&id);
+  if (!slot.ptr || !known || slot.ctx_id != id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    e = cudaGetSymbolAddress(&p, g_permute_scratch);   // also makes the primary context current
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<int*>(p);
+    slot.ptr = static_cast<int*>(p);
+    // a context the driver cannot identify is looked up again on every call
+    slot.ctx_id = current_context_id(&id) ? id : 0;
+    if (!slot.ctx_id) { *out = slot.ptr; slot.ptr = nullptr; return cudaSuccess; }
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 

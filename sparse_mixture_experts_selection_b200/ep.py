@@ -9,21 +9,21 @@ Balancing", all-to-all routing).  Shared experts run on every rank's own
 tokens; the bias step uses the loads summed over all ranks.
 
 Every step on the data runs in the library's kernels (moe_route, moe_permute,
-moe_gather_rows, moe_expert_ffn, moe_combine, moe_bias_update).  The exchange
-is the caller's: ``DistExchange`` (torch.distributed all-to-all, NCCL on GPUs)
-or ``LoopbackExchange`` (all ranks in one process, the rows moved by device
-copies -- for running and testing the whole path on one GPU).  The plan of an
-exchange (splits, regroup maps) is host arithmetic on the per-expert row
-counts of all ranks (``plan_dispatch``).
+moe_ep_plan, moe_gather_rows, moe_expert_ffn, moe_combine, moe_bias_update).
+The exchange is the caller's: ``DistExchange`` (torch.distributed: NCCL on
+device tensors; gloo through host copies) or ``LoopbackExchange`` (all ranks
+in one process, the rows moved by device copies -- for running and testing
+the whole path on one GPU).  The plan of an exchange (splits, regroup maps)
+is built on the device by moe_ep_plan from the all-gathered per-expert
+offsets; only the 2 x W split sizes are copied to the host, because the
+all-to-all takes them there.
 """
 from __future__ import annotations
 
 from dataclasses import dataclass
 from typing import List, Optional
 
-import numpy as np
-
-from . import (MoeConfig, alloc_workspace, moe_bias_update, moe_combine, moe_expert_ffn,
+from . import (MoeConfig, alloc_workspace, moe_bias_update, moe_combine, moe_ep_plan, moe_expert_ffn,
                moe_expert_ffn_workspace_size, moe_gather_rows, moe_permute, moe_route,
                moe_workspace_size)
 
@@ -32,63 +32,50 @@ from . import (MoeConfig, alloc_workspace, moe_bias_update, moe_combine, moe_exp
 class Plan:
     send_splits: List[int]      # rows this rank sends to each rank (its experts' rows of x_perm)
     recv_splits: List[int]      # rows this rank receives from each rank
-    regroup: np.ndarray         # target row -> received row (expert-major order)
-    local_offsets: np.ndarray   # [E_loc + 1] rows of each local expert after the regroup
+    regroup: "object"           # device int32 [n_recv]: regrouped row -> received row (expert-major)
+    inverse: "object"           # device int32 [n_recv]: received row -> regrouped row
+    local_offsets: "object"     # device int32 [E_loc + 1]: rows of each local expert after the regroup
     n_send: int
     n_recv: int
 
 
-def plan_dispatch(offsets_all: np.ndarray, rank: int, world: int) -> Plan:
-    """offsets_all[src] = the [E_r + 1] expert offsets of rank src's permuted rows.
-    Rows of expert e sit at offsets[e] .. offsets[e+1]; rank r owns experts
-    r*E_loc .. (r+1)*E_loc - 1, so what rank src sends to rank r is one
-    contiguous range of its rows.  Received rows arrive source by source
-    (expert-major within a source); the regroup orders them expert by expert,
-    sources ascending, each source's rows in their order."""
-    offs = np.asarray(offsets_all, np.int64)
-    E_r = offs.shape[1] - 1
-    assert E_r % world == 0, "E_r must divide evenly over the ranks"
-    E_loc = E_r // world
-    cnt = np.diff(offs, axis=1)                                    # [W, E_r]
-    lo, hi = rank * E_loc, (rank + 1) * E_loc
-    send = [int(offs[rank, (r + 1) * E_loc] - offs[rank, r * E_loc]) for r in range(world)]
-    mine = cnt[:, lo:hi]                                           # [W_src, E_loc]
-    recv = [int(x) for x in mine.sum(axis=1)]
-    local_offsets = np.concatenate([[0], np.cumsum(mine.sum(axis=0))]).astype(np.int32)
-    src_base = np.concatenate([[0], np.cumsum(recv)])[:-1]        # first received row of each source
-    regroup = np.empty(int(mine.sum()), np.int32)
-    for e in range(E_loc):
-        at = local_offsets[e]
-        for src in range(world):
-            n = int(mine[src, e])
-            first = src_base[src] + int(mine[src, :e].sum())
-            regroup[at:at + n] = np.arange(first, first + n)
-            at += n
-    return Plan(send, recv, regroup, local_offsets, int(sum(send)), int(sum(recv)))
-
-
 class DistExchange:
-    """All-to-all over torch.distributed (every rank calls the same methods)."""
+    """All-to-all over torch.distributed (every rank calls the same methods).
+    NCCL moves device tensors directly; gloo (CPU collectives) goes through
+    host copies of the same tensors."""
 
     def __init__(self, group=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
         self.world = dist.get_world_size(group)
+        self.host = dist.get_backend(group) == "gloo"
 
     # the lists hold this process's single rank (the loopback form holds all ranks)
     def all_gather_offsets(self, offs):
+        """[W, E_r + 1] int32 on offs' device: every rank's expert offsets."""
         import torch
-        out = [torch.empty_like(offs) for _ in range(self.world)]
-        self.dist.all_gather(out, offs, group=self.group)
-        return np.stack([o.cpu().numpy() for o in out])
+        src = offs.cpu() if self.host else offs
+        out = [torch.empty_like(src) for _ in range(self.world)]
+        self.dist.all_gather(out, src, group=self.group)
+        return torch.stack(out).to(offs.device)
 
     def all_to_all(self, outs, inps, out_splits, in_splits):
         (out,), (inp,), (osp,), (isp,) = outs, inps, out_splits, in_splits
-        self.dist.all_to_all_single(out, inp, list(osp), list(isp), group=self.group)
+        if self.host:
+            o = out.new_empty(out.shape, device="cpu")
+            self.dist.all_to_all_single(o, inp.cpu(), list(osp), list(isp), group=self.group)
+            out.copy_(o)
+        else:
+            self.dist.all_to_all_single(out, inp, list(osp), list(isp), group=self.group)
 
     def all_reduce_sum(self, t):
-        self.dist.all_reduce(t, group=self.group)
+        if self.host:
+            c = t.cpu()
+            self.dist.all_reduce(c, group=self.group)
+            t.copy_(c)
+        else:
+            self.dist.all_reduce(t, group=self.group)
 
 
 class ExpertParallelLayer:
@@ -106,6 +93,8 @@ class ExpertParallelLayer:
         self.E_loc = cfg.E_r // world
         self.e, self.W = e, (w_gate, w_up, w_down)
         self.WS = (ws_gate, ws_up, ws_down)
+        if cfg.dtype not in (0, 1):
+            raise ValueError(f"ExpertParallelLayer supports fp32 (0) and bf16 (1) layers, not dtype {cfg.dtype}")
         self.dt = torch.bfloat16 if cfg.dtype == 1 else torch.float32
         T, K, d = cfg.T, cfg.K, cfg.d_model
         self.ws = alloc_workspace(moe_workspace_size(cfg), device)
@@ -126,7 +115,27 @@ class ExpertParallelLayer:
         self.x_perm = torch.empty((T * K, d), dtype=self.dt, device=device)
         self.out_perm = torch.empty_like(self.x_perm)
         self.shared_out = torch.empty((max(cfg.E_s, 1), T, d), dtype=self.dt, device=device)
+        # exchange plan (moe_ep_plan): splits, local offsets, regroup and inverse maps
+        self.max_recv = max_recv
+        self.splits = torch.empty(2 * world, **i32)
+        self.local_offsets = torch.empty(self.E_loc + 1, **i32)
+        self.regroup = torch.empty(max(max_recv, 1), **i32)
+        self.inverse = torch.empty(max(max_recv, 1), **i32)
+        self.err = torch.zeros(1, **i32)
         self.device = device
+
+    # the exchange plan from every rank's offsets [W, E_r + 1] (device); the
+    # split sizes are the only values copied to the host
+    def plan(self, offsets_all) -> Plan:
+        moe_ep_plan(offsets_all, self.world, self.rank, self.cfg.E_r, self.max_recv, self.splits,
+                    self.local_offsets, self.regroup, self.inverse, self.err)
+        sp = self.splits.cpu().tolist()
+        send, recv = sp[:self.world], sp[self.world:]
+        n_recv = int(sum(recv))
+        if n_recv > self.max_recv:
+            raise RuntimeError(f"expert-parallel plan: {n_recv} rows would arrive, room for {self.max_recv}")
+        return Plan(send, recv, self.regroup[:n_recv], self.inverse[:n_recv], self.local_offsets,
+                    int(sum(send)), n_recv)
 
     # phase 1: route and permute this rank's tokens (s_in: fed fp32 scores, for tests)
     def route(self, h, b, s_in=None):
@@ -142,16 +151,13 @@ class ExpertParallelLayer:
         out_recv = torch.empty_like(x_recv)
         if n == 0:
             return out_recv
-        regroup = torch.from_numpy(plan.regroup).to(self.device)
         x_grp, g_grp = torch.empty_like(x_recv), torch.empty_like(g_recv)
-        moe_gather_rows(x_recv, n, es, regroup, n, x_grp)
-        moe_gather_rows(g_recv, n, 4, regroup, n, g_grp)
+        moe_gather_rows(x_recv, n, es, plan.regroup, n, x_grp)
+        moe_gather_rows(g_recv, n, 4, plan.regroup, n, g_grp)
         out_grp = torch.empty_like(x_recv)
-        moe_expert_ffn(self.cfg, self.E_loc, self.cfg.d_ffn, n, torch.from_numpy(plan.local_offsets).to(self.device),
+        moe_expert_ffn(self.cfg, self.E_loc, self.cfg.d_ffn, n, plan.local_offsets,
                        x_grp, self.W[0], self.W[1], self.W[2], g_grp, out_grp, self.ws_ffn)
-        inverse = np.empty_like(plan.regroup)
-        inverse[plan.regroup] = np.arange(n, dtype=np.int32)
-        moe_gather_rows(out_grp, n, es, torch.from_numpy(inverse).to(self.device), n, out_recv)
+        moe_gather_rows(out_grp, n, es, plan.inverse, n, out_recv)
         return out_recv
 
     # phase 3: shared experts, combine
@@ -176,7 +182,7 @@ def forward(layers: List[ExpertParallelLayer], hs, b, ys, exchange, gamma: float
     for i, (L, h) in enumerate(zip(layers, hs)):
         L.route(h, b, None if s_in is None else s_in[i])
     offs_all = exchange.all_gather_offsets(*[L.offsets for L in layers])
-    plans = [plan_dispatch(offs_all, L.rank, L.world) for L in layers]
+    plans = [L.plan(offs_all) for L in layers]
     d = layers[0].cfg.d_model
     x_recv = [torch.empty((p.n_recv, d), dtype=L.dt, device=L.device) for L, p in zip(layers, plans)]
     g_recv = [torch.empty(p.n_recv, dtype=torch.float32, device=L.device) for L, p in zip(layers, plans)]
@@ -207,7 +213,8 @@ class LoopbackExchange:
         self.world = world
 
     def all_gather_offsets(self, *offs):
-        return np.stack([o.cpu().numpy() for o in offs])
+        import torch
+        return torch.stack(offs)
 
     def all_to_all(self, outs, inps, out_splits, in_splits):
         W = self.world

@@ -1,6 +1,8 @@
-"""Host logic of the expert-parallel exchange (no GPU): the plan's splits and
-regroup map against a direct enumeration of the (rank, token, expert) rows,
-and the same plan computed on two gloo ranks from the gathered offsets."""
+"""Host logic of the expert-parallel exchange (no GPU): the reference plan's
+splits and regroup map (the restatement the device plan moe_ep_plan is
+compared with on the GPU) against a direct enumeration of the (rank, token,
+expert) rows, the same plan on two gloo ranks from the gathered offsets, and
+DistExchange's gloo path against the loopback exchange."""
 import os
 
 import numpy as np
@@ -10,7 +12,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from oracle import moe_oracle as mo
-from sparse_mixture_experts_selection_b200.ep import plan_dispatch
+from ep_reference import plan_reference as plan_dispatch
 
 
 def test_plan_hand_example():
@@ -105,7 +107,7 @@ def _exchange_worker(rank, world, port, q):
     try:
         rows, offs = _rank_rows(rank)
         X = DistExchange()
-        offs_all = X.all_gather_offsets(offs)
+        offs_all = X.all_gather_offsets(offs).numpy()
         plan = plan_dispatch(offs_all, rank, world)
         out = torch.empty((plan.n_recv, rows.shape[1]))
         X.all_to_all([out], [rows], [plan.recv_splits], [plan.send_splits])

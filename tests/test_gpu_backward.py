@@ -17,6 +17,7 @@ import moe_inputs as mi
 from oracle import moe_oracle as mo
 import sparse_mixture_experts_selection_b200 as moe
 import backward_cases as bc
+import bf16_backward_model as bm
 from gpu_helpers import HostWeights, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -31,6 +32,7 @@ def run_backward(w, seed=7):
     cfg_o, h, e, b, s, idx, gates, disp, dy = bc.inputs(w, seed)
     HW = HostWeights(w)
     ref = mo.layer_backward(cfg_o, h, e, s, idx, gates, disp, HW.source(), dy)
+    ref["model"] = bm.layer_backward_bf16(cfg_o, h, e, s, idx, gates, disp, HW.source(), dy)
 
     cfg = moe.config_for(w, train=1)
     Wd = HW.device()
@@ -54,13 +56,17 @@ def run_backward(w, seed=7):
 
 
 def _check_all(w, ref, dh, de, G):
+    model = ref["model"]
     bc.check(dh, ref["dh"], "dh")
+    bc.check_model(dh, model["dh"], "dh")
     if np.any(ref["de"] != 0):
         bc.check(de, ref["de"], "de")
+        bc.check_model(de, model["de"], "de")
     else:                                   # one expert: the gate is 1 whatever z is
         assert np.max(np.abs(de)) <= 1e-6
     for what, got, r in bc.each_gradient(w, ref, G):
         bc.check(got, r, what)
+        bc.check_model(got, model["grads"][what], what)
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
