@@ -643,8 +643,8 @@ def kernel_records(w, kept_h, phase_ms, ms_per_step, moe):
 
 def launches_per_step(w) -> int:
     """Our kernels per layer step: [centroid split + router GEMM | CUDA-core
-    logits], select, scan, scatter, gather (e4m3: quantize h + gather), group
-    tables, gate/up GEMM, down GEMM, combine, bias step; e4m3 adds the
+    logits], select, scan, scatter, row gather (e4m3: quantize h + gather),
+    group tables, gate/up GEMM, down GEMM, combine, bias step; e4m3 adds the
     quantization of A (and of the shared A when there are shared experts)."""
     bf16 = w.dtype != "f32"
     e4m3 = w.dtype == "bf16_e4m3"

@@ -69,7 +69,7 @@ Layout make_layout(const moe_config& c) {
   // fp32 logits: split-K partial sums of the tensor-core router (bf16 layers)
   // or the CUDA-core logits (fp32 layers)
   const bool tcr = c.dtype != MOE_DTYPE_F32;          // tensor-core router
-  L.scores = take((size_t)(tcr ? moe::kRouterMaxSplits : 1) * c.T * c.E_r * 4);
+  L.scores = take((size_t)(tcr ? moe::router_max_splits(c.T) : 1) * c.T * c.E_r * 4);
   L.e3 = take(tcr ? (size_t)3 * c.E_r * c.d_model * 2 : 0);
   L.hist = take((size_t)L.n_chunks * c.E_r * 4);
   L.chunk_base = take((size_t)L.n_chunks * c.E_r * 4);

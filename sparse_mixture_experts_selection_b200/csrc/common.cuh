@@ -101,6 +101,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The forward kernels are launched with
+// programmatic stream serialization (launch_pdl), so a kernel may start --
+// and run its prologue -- while the one before it in the stream is finishing.
+// pdl_wait blocks until that kernel has completed and its writes are visible
+// (a no-op for a kernel launched the ordinary way); every kernel calls it
+// before touching memory the previous kernels wrote, and only then lets its
+// own successor start launching (pdl_trigger), so at most one kernel waits
+// ahead.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+constexpr bool kUsePdl = true;
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// ---------------------------------------------------------------------------
 // TMA: 2-D tiled bulk tensor load global -> shared, completing on an mbarrier
 // (no multicast: each CTA loads its own tiles)
 // ---------------------------------------------------------------------------

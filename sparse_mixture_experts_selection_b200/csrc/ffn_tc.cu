@@ -46,7 +46,15 @@ constexpr int BM = 128;                         // rows per tile (MMA M)
 constexpr int BN = 256;                         // B rows per tile (MMA N)
 constexpr int BK = 64;                          // K per stage: one 128-byte swizzle atom of bf16
 constexpr int UMMA_K = 16;
-constexpr int STAGES = 4;
+// Output tiles may leave through shared memory (kernel template TMA_OUT): each
+// epilogue warp stages a 32-row x 64-column bf16 box (128-byte swizzle) and one
+// TMA tensor store writes it as whole 128-byte lines, instead of 32 threads
+// each storing 16 bytes of a different row.  The staging space (32 KB) costs
+// one stage of the operand pipeline, which long reductions feel more than
+// their stores: the launch picks it for the down GEMM when its units are short
+// (at most kTmaOutMaxKb k-blocks), where the fine-grained stores of 128 x 256
+// outputs per unit compete with the weight stream.
+constexpr int kTmaOutMaxKb = 64;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
@@ -57,18 +65,28 @@ constexpr int A_SUB_BYTES = A_SUB_ROWS * BK * 2;
 constexpr int T_BYTES = kMergeMaxRows * BK * 2; // 8 KB: a merged tail's rows per stage
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                  // 2 accumulators x 256 columns
-constexpr size_t SMEM_BYTES = (size_t)STAGES * (STAGE_BYTES + T_BYTES) + 1024 + 512;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
-constexpr uint32_t IDESC_Q8 = idesc_e4m3_f32(BM, BN);
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+constexpr int OUT_BOX_ROWS = 32;                // one epilogue warp's rows
+constexpr int OUT_BOX_BYTES = OUT_BOX_ROWS * 128;   // 32 rows x 64 bf16 columns
+constexpr int CTRL_BYTES = 512;                  // barriers and the unit ring
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1, EPI_ROUTER = 2 };
+
+// pipeline stages and shared memory with and without the output staging boxes
+template <bool TMA_OUT> constexpr int stages_of() { return TMA_OUT ? 3 : 4; }
+template <bool TMA_OUT> constexpr int out_bytes_of() { return TMA_OUT ? 4 * 2 * OUT_BOX_BYTES : 0; }
+template <bool TMA_OUT> constexpr size_t smem_of() {
+  return (size_t)stages_of<TMA_OUT>() * (STAGE_BYTES + T_BYTES) + out_bytes_of<TMA_OUT>() + 1024 + CTRL_BYTES;
+}
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC_Q8 = idesc_e4m3_f32(BM, BN);
+static_assert(smem_of<true>() <= 232448 && smem_of<false>() <= 232448, "shared memory per CTA");
 
 struct Params {
   CUtensorMap a_r, a_s;       // A: routed rows / shared rows
   CUtensorMap a32_r, a32_s;   // the same with a 32-row box (transposed tiles)
   CUtensorMap b0_r, b1_r;     // routed B: gate & up (SWIGLU) or down (b0 only)
   CUtensorMap b0_s, b1_s;     // shared B
+  CUtensorMap o_r, o_s;       // outputs (routed / shared), boxes of 32 rows x 64 columns
   const int* grp_rows;
   const int* grp_row0;
   const int* prefix;          // [G + 1] unit prefix
@@ -181,6 +199,28 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint3
   else tc_mma_bf16(d, a, b, idesc, acc);
 }
 
+// Shared -> global tensor store of one box; completion is tracked per thread
+// in bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tmap, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               :: "l"(tmap), "r"(smem_u32(smem_src)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// all but the most recent bulk group of this thread have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Write 16 bf16 pairs (32 columns) of this lane's row into the staging box:
+// line `lane`, 16-byte chunks chunk0 .. chunk0 + 3, at chunk ^ (lane & 7) --
+// the 128-byte swizzle of the store's tensor map (and bank-conflict free).
+__device__ __forceinline__ void stage_row32(uint8_t* box, int lane, int chunk0, const uint32_t (&pk)[16]) {
+  uint8_t* line = box + lane * 128;
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    *reinterpret_cast<uint4*>(line + (((chunk0 + v) ^ (lane & 7)) * 16)) =
+        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+}
+
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ uint16_t bf16_bits(float a) {
@@ -275,14 +315,18 @@ __device__ __noinline__ void epilogue_transposed(const Params& p, bool sh, uint1
 // Q8: e4m3 operands (kind::f8f6f4, epilogue scales); a template parameter so
 // that the MMA issue loop carries no branch between the two MMA forms (a
 // runtime choice there cost the bf16 kernel 15 % of its throughput).
-template <int EPI, bool Q8>
+template <int EPI, bool Q8, bool TMA_OUT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  constexpr int STAGES = stages_of<TMA_OUT>();
+  constexpr bool kTmaStoreOut = TMA_OUT && EPI != EPI_ROUTER;
+  constexpr int OUT_BYTES = out_bytes_of<TMA_OUT>();
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   uint8_t* sT = smem + STAGES * STAGE_BYTES;     // merged tails' rows
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (STAGE_BYTES + T_BYTES));
+  uint8_t* sOut = smem + STAGES * (STAGE_BYTES + T_BYTES);   // epilogue staging boxes (1024-aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -309,10 +353,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.b0_r);
     prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
     if (EPI != EPI_ROUTER) { prefetch_tmap(&p.a32_r); prefetch_tmap(&p.a32_s); }
+    if (EPI != EPI_ROUTER && kTmaStoreOut) { prefetch_tmap(&p.o_r); prefetch_tmap(&p.o_s); }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue above touches no global memory; everything below may read
+  // what the previous kernels wrote
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem_base = *tmem_slot;
   const int total = total_units<EPI>(p);
 
@@ -456,6 +505,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     uint32_t ph_f = 0;                     // bit b: phase of acc_full[b]
     int slot = 0;
     uint32_t uphase = 0;
+    uint8_t* my_boxes = sOut + sub * 2 * OUT_BOX_BYTES;   // this warp's two staging boxes
+    int n_boxes = 0;                       // boxes this warp has staged (alternating buffers)
     for (;;) {
       if (!mbar_wait(&unit_full[slot], uphase, abort_flag, p.err)) break;
       const int u = unit_ring[slot];
@@ -530,6 +581,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
                     make_float4(dv[4 * v], dv[4 * v + 1], dv[4 * v + 2], dv[4 * v + 3]);
           }
         }
+      } else if (EPI == EPI_SWIGLU && kTmaStoreOut && mt * BM + sub * 32 + 32 <= rows) {
+        // every row of this warp is valid: stage 64 columns at a time, one TMA
+        // store per box; the row stride of U | V is 2f, so those stay direct
+        const float rs = xs ? __ldg(xs + r) : 1.0f;
+        const CUtensorMap* om = sh ? &p.o_s : &p.o_r;
+        const int orow0 = (int)(orow - (size_t)lane);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 64) {
+          uint8_t* box = my_boxes + (n_boxes & 1) * OUT_BOX_BYTES;
+          if (lane == 0) bulk_wait_read_1();      // the store that last read this box is done reading
+          __syncwarp();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float gv[32], uv[32];
+            tmem_ld32(tb + c + 32 * half, gv);
+            tmem_ld32(tb + BN / 2 + c + 32 * half, uv);
+            const int col0 = nt * (BN / 2) + c + 32 * half;
+            if (xs) {
+#pragma unroll
+              for (int v = 0; v < 32; ++v) {
+                const bool in = col0 + v < ncols;
+                gv[v] *= rs * (in ? __ldg(wsA + col0 + v) : 0.0f);
+                uv[v] *= rs * (in ? __ldg(wsB + col0 + v) : 0.0f);
+              }
+            }
+            if (uv0) {
+              uint16_t* uvr = uv0 + (size_t)r * 2 * ncols;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                if (col0 + 8 * v < ncols) {
+                  *reinterpret_cast<uint4*>(uvr + col0 + 8 * v) =
+                      make_uint4(pack_bf16(gv[8 * v], gv[8 * v + 1]), pack_bf16(gv[8 * v + 2], gv[8 * v + 3]),
+                                 pack_bf16(gv[8 * v + 4], gv[8 * v + 5]), pack_bf16(gv[8 * v + 6], gv[8 * v + 7]));
+                  *reinterpret_cast<uint4*>(uvr + ncols + col0 + 8 * v) =
+                      make_uint4(pack_bf16(uv[8 * v], uv[8 * v + 1]), pack_bf16(uv[8 * v + 2], uv[8 * v + 3]),
+                                 pack_bf16(uv[8 * v + 4], uv[8 * v + 5]), pack_bf16(uv[8 * v + 6], uv[8 * v + 7]));
+                }
+              }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int v = 0; v < 16; ++v) pk[v] = pack_bf16(silu(gv[2 * v]) * uv[2 * v], silu(gv[2 * v + 1]) * uv[2 * v + 1]);
+            stage_row32(box, lane, 4 * half, pk);
+          }
+          fence_proxy_async_smem();               // the box is read by the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            const int x = nt * (BN / 2) + c;
+            if (x < ncols) tma_store_2d(om, box, x, orow0);   // columns past ncols are clipped
+            bulk_commit();                        // one group per box, even an empty one
+          }
+          ++n_boxes;
+        }
       } else if (EPI == EPI_SWIGLU) {
         const float rs = (xs && valid) ? __ldg(xs + r) : 1.0f;
 #pragma unroll 1
@@ -574,6 +678,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             }
           }
         }
+      } else if (kTmaStoreOut && mt * BM + sub * 32 + 32 <= rows) {
+        // every row of this warp is valid: stage 64 columns at a time, one TMA
+        // store per box
+        const float scale = (!sh && p.row_scale) ? __ldg(p.row_scale + orow) : 1.0f;
+        const float rs = xs ? __ldg(xs + r) : 1.0f;
+        const CUtensorMap* om = sh ? &p.o_s : &p.o_r;
+        const int orow0 = (int)(orow - (size_t)lane);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+          uint8_t* box = my_boxes + (n_boxes & 1) * OUT_BOX_BYTES;
+          if (lane == 0) bulk_wait_read_1();      // the store that last read this box is done reading
+          __syncwarp();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float dv[32];
+            tmem_ld32(tb + c + 32 * half, dv);
+            const int col0 = nt * BN + c + 32 * half;
+            if (xs) {
+#pragma unroll
+              for (int v = 0; v < 32; ++v) dv[v] *= rs * (col0 + v < ncols ? __ldg(wsA + col0 + v) : 0.0f);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int v = 0; v < 16; ++v) pk[v] = pack_bf16(dv[2 * v] * scale, dv[2 * v + 1] * scale);
+            stage_row32(box, lane, 4 * half, pk);
+          }
+          fence_proxy_async_smem();               // the box is read by the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            const int x = nt * BN + c;
+            if (x < ncols) tma_store_2d(om, box, x, orow0);   // columns past ncols are clipped
+            bulk_commit();                        // one group per box, even an empty one
+          }
+          ++n_boxes;
+        }
       } else {
         const float scale = (!sh && p.row_scale && valid) ? __ldg(p.row_scale + orow) : 1.0f;
         const float rs = (xs && valid) ? __ldg(xs + r) : 1.0f;
@@ -604,6 +743,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
+    // the staging boxes must not be released while a store still reads them
+    if (EPI != EPI_ROUTER && kTmaStoreOut && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -673,6 +814,8 @@ static int num_sms() {
 // significant bits, e_mid takes 8 of them and the last residual fits in bf16.
 __global__ void split_centroids_kernel(const float* __restrict__ e, __nv_bfloat16* __restrict__ e3,
                                        size_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
     const float x = e[i];
     const __nv_bfloat16 hi = __float2bfloat16_rn(x);
@@ -685,21 +828,31 @@ __global__ void split_centroids_kernel(const float* __restrict__ e, __nv_bfloat1
   }
 }
 
-// Split-K plan of the router GEMM: enough splits to fill the SMs, and never
-// more than kRouterMaxKbPerSplit k-blocks per split -- the tensor core's fp32
-// accumulation over long K drifts (observed 7e-6 in s at d = 7168 with 84
-// k-blocks per split), so long reductions are cut into short partial sums that
-// the select kernel adds in fp32, in split order.
+// Split-K plan of the router GEMM: never more than kRouterMaxKbPerSplit
+// k-blocks per split -- the tensor core's fp32 accumulation over long K drifts
+// (observed 7e-6 in s at d = 7168 with 84 k-blocks per split), so long
+// reductions are cut into short partial sums that the select kernel adds in
+// fp32, in split order -- and at most router_max_splits(T) splits.  Within those
+// bounds the split length minimises the modelled time, waves x (k-blocks per
+// unit + a unit's fixed cost of about kRouterUnitCostKb k-blocks) on n_sms
+// SMs; ties go to longer splits (fewer partials for the select kernel).
+constexpr int kRouterUnitCostKb = 4;
+
 void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per) {
   const int base = ((T + tc::BM - 1) / tc::BM) * ((E + tc::BN - 1) / tc::BN);
   const int total = 3 * ((d + tc::BK - 1) / tc::BK);
-  int k0 = n_sms / base;
-  k0 = k0 < 1 ? 1 : k0;
-  int p = (total + k0 - 1) / k0;
-  if (p > kRouterMaxKbPerSplit) p = kRouterMaxKbPerSplit;
-  if ((total + p - 1) / p > kRouterMaxSplits) p = (total + kRouterMaxSplits - 1) / kRouterMaxSplits;
-  *per = p;
-  *ks = (total + p - 1) / p;           // every split non-empty
+  const int max_splits = router_max_splits(T);
+  int p_lo = (total + max_splits - 1) / max_splits;
+  const int p_hi = std::max(p_lo, std::min(kRouterMaxKbPerSplit, total));
+  long best = -1;
+  int best_p = p_hi;
+  for (int p = p_hi; p >= p_lo; --p) {
+    const long units = (long)base * ((total + p - 1) / p);
+    const long t = ((units + n_sms - 1) / n_sms) * (p + kRouterUnitCostKb);
+    if (best < 0 || t < best) { best = t; best_p = p; }
+  }
+  *per = best_p;
+  *ks = (total + best_p - 1) / best_p;   // every split non-empty
 }
 
 cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpart, int T, int d,
@@ -709,12 +862,12 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_ROUTER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_ROUTER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<false>());
     attr_done[dev] = true;
   }
   const size_t n = (size_t)E * d;
-  split_centroids_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 148 * 8), 256, 0, st>>>(
-      e, reinterpret_cast<__nv_bfloat16*>(e3), n);
+  launch_pdl(split_centroids_kernel, dim3((unsigned)std::min<size_t>((n + 255) / 256, 148 * 8)), dim3(256), 0, st,
+             e, reinterpret_cast<__nv_bfloat16*>(e3), n);
   int ks, per;
   router_split_plan(T, d, E, num_sms(), &ks, &per);
   Params p{};
@@ -737,7 +890,7 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   p.err = err;
   const int units = p.r_mtiles * p.r_ntiles * ks;
   const int grid = std::min(units, num_sms());
-  grouped_gemm_kernel<EPI_ROUTER, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  launch_pdl(grouped_gemm_kernel<EPI_ROUTER, false>, dim3(grid), dim3(NUM_THREADS), smem_of<false>(), st, p);
   *ks_out = ks;
   return cudaGetLastError();
 }
@@ -748,10 +901,12 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<false>());
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<false>());
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<false>());
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<false>());
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<true>());
+    cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of<true>());
     attr_done[dev] = true;
   }
   const bool has_s = a.E_s > 0;
@@ -767,11 +922,12 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   if (which == 0) {
     // gate/up: A = permuted tokens (routed) or h (shared); B = gate | up, 128 rows each
     const uint64_t wr_r = (uint64_t)a.E_r * a.f_r, wr_s = has_s ? (uint64_t)a.E_s * a.f_s : wr_r;
-    ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM, q8);
-    ok &= make_tmap(&p.a_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d, BM, q8);
-    ok &= make_tmap(&p.a32_r, a.x_r, (uint64_t)a.max_rows_r, a.d, A_SUB_ROWS, q8);
-    ok &= make_tmap(&p.a32_s, has_s ? a.x_s : a.x_r, has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r, a.d,
-                    A_SUB_ROWS, q8);
+    const void* xr = a.x_r;
+    const uint64_t xr_rows = (uint64_t)a.max_rows_r;
+    ok &= make_tmap(&p.a_r, xr, xr_rows, a.d, BM, q8);
+    ok &= make_tmap(&p.a_s, has_s ? a.x_s : xr, has_s ? (uint64_t)a.T : xr_rows, a.d, BM, q8);
+    ok &= make_tmap(&p.a32_r, xr, xr_rows, a.d, A_SUB_ROWS, q8);
+    ok &= make_tmap(&p.a32_s, has_s ? a.x_s : xr, has_s ? (uint64_t)a.T : xr_rows, a.d, A_SUB_ROWS, q8);
     ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, BN / 2, q8);
     ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, BN / 2, q8);
     ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, BN / 2, q8);
@@ -810,6 +966,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
       p.s0_r = p.s1_r = blob_scales(a.wd_r, (uint64_t)a.E_r * a.d, a.f_r);
       p.s0_s = p.s1_s = has_s ? blob_scales(a.wd_s, wd_rows_s, fs) : p.s0_r;
     }
+    ok &= make_tmap(&p.o_r, a.out_r, (uint64_t)a.max_rows_r, a.d, OUT_BOX_ROWS);
+    ok &= make_tmap(&p.o_s, has_s ? a.out_s : a.out_r, rows_s, a.d, OUT_BOX_ROWS);
     p.prefix = a.pre_dn;
     p.k_r = a.f_r; p.k_s = a.f_s;
     p.wrows_r = a.d; p.wrows_s = a.d;
@@ -820,15 +978,15 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   if (!ok) return cudaErrorInvalidValue;
   p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
   const int grid = num_sms();
-  if (which == 0 && q8)
-    grouped_gemm_kernel<EPI_SWIGLU, true><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
-  else if (which == 0)
-    grouped_gemm_kernel<EPI_SWIGLU, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
-  else if (q8)
-    grouped_gemm_kernel<EPI_SCALE, true><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
-  else
-    grouped_gemm_kernel<EPI_SCALE, false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
-  return cudaGetLastError();
+  // down GEMM with short units: outputs through the staging boxes and TMA stores
+  const int kb_r = (a.f_r + p.bk - 1) / p.bk, kb_s = (p.k_s + p.bk - 1) / p.bk;
+  const bool tma_out = which == 1 && std::max(kb_r, has_s ? kb_s : 0) <= kTmaOutMaxKb;
+  auto kern = which == 0 ? (q8 ? grouped_gemm_kernel<EPI_SWIGLU, true> : grouped_gemm_kernel<EPI_SWIGLU, false>)
+            : tma_out ? (q8 ? grouped_gemm_kernel<EPI_SCALE, true, true> : grouped_gemm_kernel<EPI_SCALE, false, true>)
+                      : (q8 ? grouped_gemm_kernel<EPI_SCALE, true> : grouped_gemm_kernel<EPI_SCALE, false>);
+  const size_t smem = tma_out ? smem_of<true>() : smem_of<false>();
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(NUM_THREADS), smem, st, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -82,8 +82,16 @@ void launch_ffn_simt(const FfnArgs& a, int which, cudaStream_t st);
 // Router logits on the tensor cores: split e into three bf16 terms (e3 =
 // [3, E, d] bf16 scratch) and write fp32 partial logits zpart [ks, T, E] over
 // ks split-K ranges (summed in order by the select kernel).
+// At most kRouterMaxSplits partials (kRouterMaxSplitsSmallT for batches of
+// at most kRouterSmallT tokens, where one row tile leaves most SMs idle unless
+// the reduction is cut finer); the select kernel adds them kRouterPartChunk
+// at a time.
 constexpr int kRouterMaxSplits = 16;
+constexpr int kRouterMaxSplitsSmallT = 64;
+constexpr int kRouterSmallT = 1024;
+constexpr int kRouterPartChunk = 16;
 constexpr int kRouterMaxKbPerSplit = 24;
+inline int router_max_splits(int T) { return T <= kRouterSmallT ? kRouterMaxSplitsSmallT : kRouterMaxSplits; }
 void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per);
 cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpart, int T, int d,
                              int E, int* err, int* ks_out, cudaStream_t st);

@@ -88,6 +88,8 @@ select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const
               int score_fn, float* __restrict__ s_out, float* __restrict__ z_out, int32_t* __restrict__ idx,
               float* __restrict__ gates, int* __restrict__ hist, int chunk_shift, int T, int E,
               int K, int n_groups, int topk_groups, int group_topn) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
   if (t >= T) return;
@@ -97,10 +99,21 @@ select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const
 #pragma unroll
   for (int j = 0; j < KPL; ++j) {
     int ex = j * kWarp + lane;
-    s[j] = ex < E ? row[ex] : 0.f;
-    // logits from split-K partial sums: added in split order (deterministic)
-    for (int q = 1; q < n_parts; ++q)
-      if (ex < E) s[j] = __fadd_rn(s[j], row[(size_t)q * T * E + ex]);
+    // logits from split-K partial sums: the partials are loaded
+    // kRouterPartChunk at a time (all loads of a chunk in flight together)
+    // and added in split order (deterministic)
+    float acc = 0.f;
+    for (int q0 = 0; q0 < n_parts; q0 += kRouterPartChunk) {
+      float part[kRouterPartChunk];
+#pragma unroll
+      for (int q = 0; q < kRouterPartChunk; ++q)
+        part[q] = (q0 + q < n_parts && ex < E) ? row[(size_t)(q0 + q) * T * E + ex] : 0.f;
+      acc = q0 == 0 ? part[0] : __fadd_rn(acc, part[0]);
+#pragma unroll
+      for (int q = 1; q < kRouterPartChunk; ++q)
+        if (q0 + q < n_parts) acc = __fadd_rn(acc, part[q]);
+    }
+    s[j] = ex < E ? acc : 0.f;
   }
   if (!in_is_scores) {
     if (z_out) {
@@ -312,6 +325,8 @@ __device__ int block_exclusive_scan(int v, int* total) {
 __global__ void __launch_bounds__(1024)
 scan_kernel(const int* __restrict__ hist, int n_chunks, int E, int cap, int* __restrict__ counts,
             int* __restrict__ kept, int* __restrict__ offsets, int* __restrict__ chunk_base) {
+  pdl_wait();
+  pdl_trigger();
   const int ex = threadIdx.x;
   int kv = 0;
   if (ex < E) {
@@ -340,6 +355,8 @@ groups_kernel(const int* __restrict__ offsets, int E_r, int E_s, int T, int bm, 
               int nt_gu_s, int nt_dn_r, int nt_dn_s, int* __restrict__ grp_rows,
               int* __restrict__ grp_row0, int* __restrict__ pre_gu, int* __restrict__ pre_dn,
               int max_rows, int* err, int* tile_counters) {
+  pdl_wait();
+  pdl_trigger();
   if (tile_counters && threadIdx.x < 2) tile_counters[threadIdx.x] = 0;   // GEMM unit counters
   const int G = E_r + E_s;
   // routed offsets must be non-decreasing within [0, max_rows]; otherwise no
@@ -385,6 +402,8 @@ scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gates,
                const int* __restrict__ offsets, const int* __restrict__ chunk_base, int cap,
                int T, int K, int E, int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of,
                float* __restrict__ row_gate, int* err) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint32_t sm_scatter[];
   uint32_t* wmask = sm_scatter;                        // [8][E]
   int* wbase = reinterpret_cast<int*>(sm_scatter + 8 * E);   // [8][E]
@@ -436,6 +455,8 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* _
                                    const int* __restrict__ n_rows_ptr, uint4* __restrict__ x_perm,
                                    int vec_per_row, int n_tok, int max_rows, int* err,
                                    const float* __restrict__ s_src, float* __restrict__ s_dst) {
+  pdl_wait();
+  pdl_trigger();
   const int n = min(*n_rows_ptr, max_rows);
   const int lane = threadIdx.x % kWarp;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
@@ -490,6 +511,8 @@ __global__ void __launch_bounds__(128)
 combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
                const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int K,
                int E_s, int add_residual, int n_slot_rows) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
   int rows[32];
@@ -536,6 +559,8 @@ __global__ void __launch_bounds__(128)
 combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
                  const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int E_s,
                  int add_residual, int n_slot_rows) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
   int rows[KT];
@@ -582,6 +607,8 @@ combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* _
 __global__ void __launch_bounds__(1024)
 bias_update_kernel(const int* __restrict__ counts, float* __restrict__ b, float gamma,
                    float* __restrict__ max_vio, int E, int K, int T) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int smax[32];
   const int ex = threadIdx.x;
   int c = ex < E ? counts[ex] : 0;
@@ -770,8 +797,8 @@ void launch_select(const float* in, int n_parts, int in_is_scores, const float* 
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps);
   int kpl = (E + 31) / 32;
-#define MOE_SEL(N) select_kernel<N><<<grid, warps * 32, 0, st>>>(in, n_parts, in_is_scores, bias, score_fn, \
-      s_out, z_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
+#define MOE_SEL(N) launch_pdl(select_kernel<N>, grid, dim3(warps * 32), 0, st, in, n_parts, in_is_scores, bias, \
+      score_fn, s_out, z_out, idx, gates, hist, chunk_shift, T, E, K, n_groups, topk_groups, group_topn)
   if (kpl <= 1) MOE_SEL(1);
   else if (kpl <= 2) MOE_SEL(2);
   else if (kpl <= 4) MOE_SEL(4);
@@ -793,14 +820,14 @@ void launch_counts(const int* hist, int n_chunks, int E, int* counts, cudaStream
 
 void launch_scan(const int* hist, int n_chunks, int E, int cap, int* counts, int* kept,
                  int* offsets, int* chunk_base, cudaStream_t st) {
-  scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, cap, counts, kept, offsets, chunk_base);
+  launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, hist, n_chunks, E, cap, counts, kept, offsets, chunk_base);
 }
 
 void launch_groups(const int* offsets, int E_r, int E_s, int T, int bm, int merge_max, int nt_gu_r, int nt_gu_s,
                    int nt_dn_r, int nt_dn_s, int* grp_rows, int* grp_row0, int* pre_gu,
                    int* pre_dn, int max_rows, int* err, int* tile_counters, cudaStream_t st) {
-  groups_kernel<<<1, 1024, 0, st>>>(offsets, E_r, E_s, T, bm, merge_max, nt_gu_r, nt_gu_s, nt_dn_r, nt_dn_s,
-                                    grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err, tile_counters);
+  launch_pdl(groups_kernel, dim3(1), dim3(1024), 0, st, offsets, E_r, E_s, T, bm, merge_max, nt_gu_r, nt_gu_s,
+             nt_dn_r, nt_dn_s, grp_rows, grp_row0, pre_gu, pre_dn, max_rows, err, tile_counters);
 }
 
 void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
@@ -815,8 +842,8 @@ void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
     cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 16 * 1024 * 4);
     attr_done[dev] = true;
   }
-  scatter_kernel<<<n_chunks, 256, smem, st>>>(idx, gates, offsets, chunk_base, cap, T, K, E,
-                                              perm_tok, row_of, row_gate, err);
+  launch_pdl(scatter_kernel, dim3(n_chunks), dim3(256), smem, st, idx, gates, offsets, chunk_base, cap, T, K, E,
+             perm_tok, row_of, row_gate, err);
 }
 
 void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
@@ -826,8 +853,8 @@ void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr
   int warps = max_rows < 148 * 64 ? max_rows : 148 * 64;
   if (warps < 1) warps = 1;
   int blocks = (warps * 32 + 255) / 256;
-  gather_rows_kernel<<<blocks, 256, 0, st>>>((const uint4*)h, perm_tok, n_rows_ptr, (uint4*)x_perm,
-                                             vec, n_tok, max_rows, err, s_src, s_dst);
+  launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, (const uint4*)h, perm_tok, n_rows_ptr,
+             (uint4*)x_perm, vec, n_tok, max_rows, err, s_src, s_dst);
 }
 
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
@@ -842,17 +869,15 @@ void launch_combine(const void* h, const void* slot, const void* shared, const i
   if (dtype == MOE_DTYPE_BF16 && (K == 2 || K == 4 || K == 6 || K == 8)) {
     const bf16 *hh = (const bf16*)h, *sl = (const bf16*)slot, *sh = (const bf16*)shared;
     bf16* yy = (bf16*)y;
-    if (K == 8) combine_k_kernel<bf16, 8><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
-    else if (K == 6) combine_k_kernel<bf16, 6><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
-    else if (K == 4) combine_k_kernel<bf16, 4><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
-    else combine_k_kernel<bf16, 2><<<grid, 128, 0, st>>>(hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+    auto kern = K == 8 ? combine_k_kernel<bf16, 8> : K == 6 ? combine_k_kernel<bf16, 6>
+              : K == 4 ? combine_k_kernel<bf16, 4> : combine_k_kernel<bf16, 2>;
+    launch_pdl(kern, grid, dim3(128), 0, st, hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
   } else if (dtype == MOE_DTYPE_BF16)
-    combine_kernel<bf16><<<grid, 128, 0, st>>>((const bf16*)h, (const bf16*)slot, (const bf16*)shared,
-                                            row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
+    launch_pdl(combine_kernel<bf16>, grid, dim3(128), 0, st, (const bf16*)h, (const bf16*)slot, (const bf16*)shared,
+               row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
   else
-    combine_kernel<float><<<grid, 128, 0, st>>>((const float*)h, (const float*)slot,
-                                             (const float*)shared, row_of, (float*)y, T, d, K, E_s,
-                                             add_residual, n_slot_rows);
+    launch_pdl(combine_kernel<float>, grid, dim3(128), 0, st, (const float*)h, (const float*)slot,
+               (const float*)shared, row_of, (float*)y, T, d, K, E_s, add_residual, n_slot_rows);
 }
 
 void launch_gather_map(const void* src, const int32_t* map, int64_t n_rows, int64_t n_src, int row_bytes,
@@ -865,7 +890,7 @@ void launch_gather_map(const void* src, const int32_t* map, int64_t n_rows, int6
 
 void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
                         int T, cudaStream_t st) {
-  bias_update_kernel<<<1, 1024, 0, st>>>(counts, b, gamma, max_vio, E, K, T);
+  launch_pdl(bias_update_kernel, dim3(1), dim3(1024), 0, st, counts, b, gamma, max_vio, E, K, T);
 }
 
 }  // namespace moe

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     for s in syms:
         assert hasattr(L, s), s
     assert set(syms) == set(moe.SIGNATURES), set(syms) ^ set(moe.SIGNATURES)
-    assert L.moe_abi_version() == 2
+    assert L.moe_abi_version() == 3
     assert moe.lib().moe_status_string(3) == b"MOE_ERR_WORKSPACE"
 
 
@@ -122,6 +122,15 @@ def test_entry_points_validate_pointers_before_any_launch():
     assert L.moe_expert_ffn_workspace_size(ctypes.byref(c), 8, 128, 10, ctypes.byref(n)) == 0
     assert L.moe_expert_ffn(ctypes.byref(c), 8, 128, 10, P, P, P, P, P, None, P, P, n.value - 1, None) == 3
     assert L.moe_get_device_error(None, None) == 1
+    # expert-parallel plan: world, rank and the expert split are checked before any launch
+    assert L.moe_ep_plan(P, 0, 0, 16, 10, P, P, P, P, None, None) == 1          # world < 1
+    assert L.moe_ep_plan(P, 65, 0, 65 * 4, 10, P, P, P, P, None, None) == 1     # world > 64
+    assert L.moe_ep_plan(P, 4, 4, 16, 10, P, P, P, P, None, None) == 1          # rank >= world
+    assert L.moe_ep_plan(P, 3, 0, 16, 10, P, P, P, P, None, None) == 1          # E_r % world
+    assert L.moe_ep_plan(P, 4, 0, 2048, 10, P, P, P, P, None, None) == 1        # E_r > 1024
+    assert L.moe_ep_plan(P, 4, 0, 16, -1, P, P, P, P, None, None) == 1          # max_recv < 0
+    assert L.moe_ep_plan(P, 4, 0, 16, 10, P, P, None, P, None, None) == 1       # regroup NULL
+    assert L.moe_ep_plan(P + 2, 4, 0, 16, 10, P, P, P, P, None, None) == 1      # misaligned offsets
     # router statistics: seq_len must divide T; stats required
     n = ctypes.c_size_t(0)
     assert L.moe_router_stats_workspace_size(ctypes.byref(c), 7, ctypes.byref(n)) == 1
