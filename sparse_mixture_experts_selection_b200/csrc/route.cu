@@ -553,9 +553,12 @@ combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __r
 // Combine with K fixed at compile time: the K row indices stay in registers
 // and every row's 16-byte chunk is loaded before the sums, which run in the
 // same fixed order as combine_kernel (h, shared j ascending, slots k
-// ascending), so the results are bit-identical.
+// ascending), so the results are bit-identical.  Six resident blocks per SM
+// (registers capped at 80): more loads in flight per SM than the five the
+// unconstrained register count allows (measured 10-12 % faster), without the
+// spills that eight would cost.
 template <typename T, int KT>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 6)
 combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
                  const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int E_s,
                  int add_residual, int n_slot_rows) {
