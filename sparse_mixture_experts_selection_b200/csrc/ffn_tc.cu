@@ -392,6 +392,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
           const TileCoords<EPI> c = tile_coords<EPI>(p, w, i);
           mbar_arrive_expect_tx(&full[stage], tx);
+          // the weight tile first: it comes from HBM, the row tiles mostly from L2
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
+            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, c.b1, &full[stage], c.bx, c.by);
+          } else {
+            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
+          }
           if (n_sub == 0) {
             tma_load_2d(sA + stage * A_BYTES, c.am, &full[stage], c.ax, c.ay);
           } else {
@@ -402,12 +409,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           for (int q = 0; q < t_sub; ++q)
             tma_load_2d(sT + stage * T_BYTES + q * A_SUB_BYTES, c.am32, &full[stage], c.ax,
                         c.ay + BM + q * A_SUB_ROWS);
-          if (EPI == EPI_SWIGLU) {
-            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
-            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, c.b1, &full[stage], c.bx, c.by);
-          } else {
-            tma_load_2d(sB + stage * B_BYTES, c.b0, &full[stage], c.bx, c.by);
-          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
