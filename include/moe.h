@@ -186,6 +186,10 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* idx, const float* g
  *   out          [max_rows, d], cfg->dtype.  Rows >= offsets[n_experts] untouched.
  * bf16 runs on the tensor cores (tcgen05, fp32 accumulation in TMEM; the SwiGLU
  * product is rounded to bf16 before W_down); fp32 runs on CUDA cores in fp32.
+ * bf16 inference with max_rows >= 512 * n_experts (many rows per expert, as in
+ * a dropless layer with T*K/E_r >= 512) runs both GEMMs on CTA pairs (clusters
+ * of two CTAs, tcgen05 cta_group::2, 256-row tiles): the same arithmetic, with
+ * the tensor core's own summation order inside each 16-element step.
  */
 /* Workspace bytes moe_expert_ffn needs for these arguments (*bytes: HOST pointer). */
 moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,

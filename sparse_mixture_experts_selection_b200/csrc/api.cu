@@ -229,10 +229,16 @@ void mark_phase(int i, cudaStream_t st) {
 moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int max_rows,
                    cudaStream_t st, int phase_base = -1) {
   const bool tc = use_tensor_cores(c.dtype);
-  const int bm = tc ? moe::tc_bm() : moe::simt_bm();
+  // bf16 inference layers whose experts average many rows (the rows the
+  // caller provisions per routed expert: T*K/E_r in a dropless layer) run
+  // their GEMMs on CTA pairs (256-row tiles); the group tables follow that
+  // tile height
+  a.pair = tc && !a.q8 && a.uv_r == nullptr && a.E_r > 0 &&
+           (int64_t)max_rows >= (int64_t)moe::tc_pair_min_rows() * a.E_r;
+  const int bm = a.pair ? moe::tc_pair_rows() : tc ? moe::tc_bm() : moe::simt_bm();
   const int bn_gu = tc ? moe::tc_cols_gateup() : moe::simt_bn();
   const int bn_dn = tc ? moe::tc_cols_down() : moe::simt_bn();
-  moe::launch_groups(offsets, a.E_r, a.E_s, a.T, bm, tc ? moe::tc_merge_rows() : 0, (a.f_r + bn_gu - 1) / bn_gu,
+  moe::launch_groups(offsets, a.E_r, a.E_s, a.T, bm, a.pair ? moe::tc_pair_merge_rows() : tc ? moe::tc_merge_rows() : 0, (a.f_r + bn_gu - 1) / bn_gu,
                      a.E_s ? (a.f_s + bn_gu - 1) / bn_gu : 0, (a.d + bn_dn - 1) / bn_dn,
                      (a.d + bn_dn - 1) / bn_dn, const_cast<int*>(a.grp_rows),
                      const_cast<int*>(a.grp_row0), const_cast<int*>(a.pre_gu),

@@ -755,6 +755,507 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair grouped GEMM (tcgen05 cta_group::2) for experts with many rows.
+//
+// A cluster of two CTAs on neighbouring SMs computes 256-row x 256-column
+// tiles: each CTA stages its own 128 rows of A and one half of the weight tile,
+// and one thread of the even CTA issues M = 256 MMAs that read both CTAs'
+// shared memory and accumulate each CTA's 128 rows in its own TMEM.  Per SM a
+// k-block then costs 32 KB of operands for the same tensor work as a 48 KB
+// stage of the single-CTA kernel, so six stages fit and each weight tile
+// crosses L2 -> SM once per 256 rows instead of once per 128.
+//
+// Weight halves: for the down GEMM the even CTA holds rows 0..127 of W_down's
+// 256-row tile and the odd CTA rows 128..255; for the gate/up GEMM each CTA
+// holds 64 gate rows and the 64 up rows of the same output columns (the even
+// CTA columns 0..63 of the 128-column tile, the odd CTA 64..127), so the
+// accumulator columns are [gate 0..63 | up 0..63 | gate 64..127 | up 64..127].
+//
+// Merged tails: a group's last tile of at most kPairMergeMax rows rides in the
+// unit of the full tile before it.  Each CTA stages half of the tail's rows,
+// and one more MMA per k-step computes the tail transposed, D^T = W x^T with
+// the two staged weight halves as the M = 256 operand and the tail rows as the
+// N = round16(tail) operand, into the second accumulator: TMEM lane = weight
+// row, column = tail row.  For the gate/up GEMM the gate rows land in lanes
+// 0..63 and the up rows of the same columns in lanes 64..127 of the same CTA;
+// the epilogue warps exchange them through shared memory.  Other short last
+// tiles are padded to 256 rows, so the launch takes this kernel only when
+// experts average many rows (kPairMinRows).  Units are claimed dynamically by
+// the even CTA's producer (merged units cost more than plain ones, so a fixed
+// round-robin leaves some pairs with more work) and handed to both CTAs through
+// a unit ring mirrored in each CTA's shared memory.
+//
+// Barriers: full[s] lives in the even CTA and counts both CTAs' TMA bytes
+// (the even CTA arms it with both halves; the odd CTA's loads complete on it
+// through its cluster address); empty[s] and acc_full[a] exist in both CTAs
+// and are signalled together by one multicast commit; acc_empty[a] lives in
+// the even CTA and takes one arrival per epilogue warp of both CTAs.  Unit
+// ring: the even CTA's producer writes each claimed unit into slot s of both
+// CTAs (the odd CTA's by a remote store followed by a release arrive on its
+// unit_full[s]); unit_empty[s] lives in the even CTA and takes one arrival
+// from each reader: the MMA thread, the producer of the odd CTA and every
+// epilogue warp of both CTAs.
+// ---------------------------------------------------------------------------
+constexpr int kPairMinRows = 512;               // routed rows per expert (mean) for the pair kernel
+constexpr int kPairMergeMax = 64;               // tails of <= this many rows join the tile before
+constexpr int P_M = 2 * BM;                     // 256 rows per pair tile
+constexpr int P_B_BYTES = (BN / 2) * BK * 2;    // 16 KB: this CTA's half of the weight tile
+constexpr int P_T_BYTES = A_SUB_BYTES;          // 4 KB: a 32-row box of this CTA's tail rows
+constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES + P_T_BYTES;
+constexpr int P_STAGES = 6;
+constexpr int P_XCHG_BYTES = 32 * 64 * 4;       // 8 KB: up values of 32 tail rows x 64 columns
+constexpr size_t P_SMEM = (size_t)P_STAGES * P_STAGE_BYTES + P_XCHG_BYTES + 1024 + CTRL_BYTES;
+constexpr uint32_t P_IDESC = idesc_bf16_f32(P_M, BN);
+static_assert(P_SMEM <= 232448, "shared memory per CTA");
+static_assert(kPairMergeMax <= 2 * A_SUB_ROWS, "a tail's half fits one 32-row box");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared-memory location in cluster CTA `rank`
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void st_remote_u32(uint32_t addr_cluster, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+// the four epilogue warps of this CTA (named barrier 1; __syncthreads uses 0)
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// TMA load into this CTA's shared memory, its bytes counted on the barrier at
+// cluster address bar_cluster (the even CTA's); no multicast
+__device__ __forceinline__ void tma_load_2d_pair(void* sdst, const void* tmap, uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(sdst)), "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+// arrive on `bar` in both CTAs of the pair once this thread's MMAs are done
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(smem_u32(bar)), "h"((uint16_t)3) : "memory");
+}
+// arrive on `bar` in this CTA only
+__device__ __forceinline__ void tc_commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(smem_slot)), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// One unit of the pair kernel: group g, 256-row tile mt, column tile nt; tail
+// > 0 marks a full tile carrying the group's last `tail` rows (t16 rounded up
+// to 16) as its merged tail.
+struct PairUnit {
+  int g, mt, nt, nk, rows, tail, t16;
+  bool sh;
+};
+
+__device__ __forceinline__ PairUnit pair_decode(const Params& p, int u) {
+  PairUnit w;
+  int lo = 0, hi = p.G;                  // prefix[lo] <= u < prefix[lo + 1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.prefix + mid) <= u) lo = mid; else hi = mid;
+  }
+  w.g = lo;
+  w.sh = lo >= p.E_r;
+  const int local = u - __ldg(p.prefix + lo);
+  w.rows = __ldg(p.grp_rows + lo);
+  const int mtiles = (w.rows + P_M - 1) / P_M;
+  const int last = w.rows - (mtiles - 1) * P_M;
+  const int runits = mtiles - ((mtiles >= 2 && last <= kPairMergeMax) ? 1 : 0);
+  w.mt = local % runits;
+  w.nt = local / runits;
+  w.tail = (runits < mtiles && w.mt == runits - 1) ? last : 0;
+  w.t16 = (w.tail + 15) & ~15;
+  w.nk = ((w.sh ? p.k_s : p.k_r) + p.bk - 1) / p.bk;
+  return w;
+}
+
+// A bounded wait that also tells the other CTA of the pair to give up.
+__device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                          uint32_t peer_abort) {
+  if (mbar_wait(bar, parity, abort, err)) return true;
+  st_remote_u32(peer_abort, 1u);
+  return false;
+}
+
+// The same with acquire semantics at cluster scope: for the unit ring, whose
+// slots the other CTA writes (remote store, then a release arrive).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool pair_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                                  uint32_t peer_abort) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 63u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        set_device_error(err, MOE_DEVERR_WAIT_TIMEOUT);
+        *abort = 1;
+        st_remote_u32(peer_abort, 1u);
+        return false;
+      }
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + P_STAGES * A_BYTES;
+  uint8_t* sT = sB + P_STAGES * P_B_BYTES;
+  float* xchg = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES + P_XCHG_BYTES);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* acc_full = empty + P_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* unit_full = drain + 1;
+  uint64_t* unit_empty = unit_full + UNIT_RING;
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(unit_empty + UNIT_RING);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UNIT_RING);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  constexpr int kUnitReaders = 1 + 1 + 2 * 4;   // MMA thread, odd producer, epilogue warps
+
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer_abort = cluster_addr(const_cast<int*>(abort_flag), rank ^ 1u);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 2 * 4); }
+    for (int s = 0; s < UNIT_RING; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], kUnitReaders); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.a32_r); prefetch_tmap(&p.a32_s);
+    prefetch_tmap(&p.b0_r); prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
+  }
+  __syncthreads();
+  cluster_sync_all();          // both CTAs' barriers are initialised before either signals the other
+  if (warp == 0) tmem_alloc_pair(tmem_slot, TMEM_COLS);   // the same warp in both CTAs
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = __ldg(p.prefix + p.G);
+  const int pair = (int)blockIdx.x >> 1, n_pairs = (int)gridDim.x >> 1;
+  const uint32_t leader_unit_empty = cluster_addr(unit_empty, 0);   // slot s: + 8 s
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int slot = 0;
+      uint32_t uphase = 0;
+      int n_claims = 0;
+      for (;;) {
+        int u;
+        if (rank == 0) {
+          // claim the next unit and hand it to both CTAs (-1 = done)
+          u = p.tile_counter ? atomicAdd(p.tile_counter, 1) : pair + n_claims * n_pairs;
+          ++n_claims;
+          if (u >= total) u = -1;
+          if (!pair_wait_cluster(&unit_empty[slot], uphase ^ 1u, abort_flag, p.err, peer_abort)) goto producer_done;
+          unit_ring[slot] = u;
+          st_remote_u32(cluster_addr(const_cast<int*>(unit_ring + slot), 1), (uint32_t)u);
+          mbar_arrive(&unit_full[slot]);
+          mbar_arrive_remote(cluster_addr(&unit_full[slot], 1));
+        } else {
+          if (!pair_wait_cluster(&unit_full[slot], uphase, abort_flag, p.err, peer_abort)) goto producer_done;
+          u = unit_ring[slot];
+          mbar_arrive_remote(leader_unit_empty + 8u * slot);
+        }
+        if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+        if (u < 0) break;
+        const PairUnit w = pair_decode(p, u);
+        const int e = w.sh ? w.g - p.E_r : w.g;
+        const CUtensorMap* am = w.sh ? &p.a_s : &p.a_r;
+        const CUtensorMap* am32 = w.sh ? &p.a32_s : &p.a32_r;
+        const int row_base = (EPI == EPI_SWIGLU && w.sh) ? 0 : __ldg(p.grp_row0 + w.g);
+        const int ay = row_base + w.mt * P_M + (int)rank * BM;
+        // this CTA's half of the merged tail: rows rank * t16/2 .. of the tail
+        const int ty = row_base + (w.mt + 1) * P_M + (int)rank * (w.t16 / 2);
+        const int wrows = w.sh ? p.wrows_s : p.wrows_r;
+        const CUtensorMap* b0 = w.sh ? &p.b0_s : &p.b0_r;
+        const CUtensorMap* b1 = w.sh ? &p.b1_s : &p.b1_r;
+        const int by = EPI == EPI_SWIGLU ? e * wrows + w.nt * (BN / 2) + (int)rank * (BN / 4)
+                                         : e * wrows + w.nt * BN + (int)rank * (BN / 2);
+        const uint32_t tx = 2u * (A_BYTES + P_B_BYTES + (w.tail ? P_T_BYTES : 0));
+        for (int i = 0; i < w.nk; ++i) {
+          if (!pair_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, peer_abort)) goto producer_done;
+          const uint32_t bar = cluster_addr(&full[stage], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx);
+          const int x = i * p.bk;
+          if (EPI == EPI_SWIGLU) {
+            // 64 gate rows, then the 64 up rows of the same columns
+            tma_load_2d_pair(sB + stage * P_B_BYTES, b0, bar, x, by);
+            tma_load_2d_pair(sB + stage * P_B_BYTES + P_B_BYTES / 2, b1, bar, x, by);
+          } else {
+            tma_load_2d_pair(sB + stage * P_B_BYTES, b0, bar, x, by);
+          }
+          tma_load_2d_pair(sA + stage * A_BYTES, am, bar, x, ay);
+          if (w.tail) tma_load_2d_pair(sT + stage * P_T_BYTES, am32, bar, x, ty);
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // every stage's last release (the MMA commits reach both CTAs) has
+      // arrived before this CTA may leave
+      for (int i = 0; i < P_STAGES; ++i) {
+        if (!pair_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, peer_abort)) break;
+        if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (even CTA) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int nb = 0;                           // accumulator of the next one-buffer unit
+      uint32_t ph_e = 0;                    // bit a: phase of acc_empty[a]
+      bool ok = true;
+      int slot = 0;
+      uint32_t uphase = 0;
+      for (;;) {
+        if (!pair_wait(&unit_full[slot], uphase, abort_flag, p.err, peer_abort)) { ok = false; break; }
+        const int u = unit_ring[slot];
+        mbar_arrive(&unit_empty[slot]);
+        if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+        if (u < 0) break;
+        const PairUnit w = pair_decode(p, u);
+        // a unit with a merged tail holds accumulator 0 (full tile) and 1 (tail)
+        const bool two = w.tail > 0;
+        const int acc = two ? 0 : nb;
+        if (!pair_wait(&acc_empty[acc], ((ph_e >> acc) & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
+        ph_e ^= 1u << acc;
+        if (two) {
+          if (!pair_wait(&acc_empty[1], ((ph_e >> 1) & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
+          ph_e ^= 2u;
+        }
+        nb = two ? 1 : nb ^ 1;              // after a merged unit, the tail's buffer frees first
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tail = tmem_base + (uint32_t)BN;
+        const uint32_t idesc_tail = idesc_bf16_f32(P_M, w.t16 ? w.t16 : 16);
+        for (int kb = 0; kb < w.nk; ++kb) {
+          if (!pair_wait(&full[stage], phase, abort_flag, p.err, peer_abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * P_B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            tc_mma_pair(d_tmem, sdesc_kmajor_sw128(a0 + k * UMMA_K * 2), sdesc_kmajor_sw128(b0 + k * UMMA_K * 2),
+                        P_IDESC, (kb | k) != 0);
+          if (two) {
+            const uint32_t t0 = smem_u32(sT + stage * P_T_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              tc_mma_pair(d_tail, sdesc_kmajor_sw128(b0 + k * UMMA_K * 2), sdesc_kmajor_sw128(t0 + k * UMMA_K * 2),
+                          idesc_tail, (kb | k) != 0);
+          }
+          tc_commit_pair(&empty[stage]);    // frees the stage in both CTAs once these MMAs are done
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(&acc_full[acc]);     // both CTAs' halves of the accumulator are ready
+        if (two) tc_commit_pair(&acc_full[1]);
+      }
+      // the epilogues of both CTAs have released both accumulators
+      for (int a = 0; a < 2 && ok; ++a)
+        if (!pair_wait(&acc_empty[a], ((ph_e >> a) & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
+      tc_commit_local(drain);               // every MMA issued by this thread is done
+      wait_drain(drain, 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int sub = warp & 3;              // TMEM lane quarter this warp may access
+    const int L = sub * 32 + lane;         // this thread's TMEM lane
+    int nb = 0;
+    uint32_t ph_f = 0;
+    int slot = 0;
+    uint32_t uphase = 0;
+    for (;;) {
+      if (!pair_wait_cluster(&unit_full[slot], uphase, abort_flag, p.err, peer_abort)) break;
+      const int u = unit_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_unit_empty + 8u * slot);
+      if (++slot == UNIT_RING) { slot = 0; uphase ^= 1u; }
+      if (u < 0) break;
+      const PairUnit w = pair_decode(p, u);
+      const bool two = w.tail > 0;
+      const int acc = two ? 0 : nb;
+      nb = two ? 1 : nb ^ 1;
+      const int ncols = w.sh ? p.ncols_s : p.ncols_r;
+      uint16_t* outb = w.sh ? p.out_s : p.out_r;
+      const size_t grow0 = (size_t)__ldg(p.grp_row0 + w.g);      // output row of group row 0
+      if (two) {
+        // the merged tail (group rows (mt + 1) * 256 ..), transposed, accumulator 1
+        // first: its buffer is the one the next unit takes
+        if (!pair_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err, peer_abort)) break;
+        ph_f ^= 2u;
+        tc_fence_after();
+        const size_t trow0 = grow0 + (size_t)(w.mt + 1) * P_M;
+        const uint32_t tt = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN;
+        for (int c = 0; c < w.t16; c += 32) {
+          float dv[32];
+          if (EPI == EPI_SWIGLU) {
+            // lanes 64..127 hold up; hand them to the gate lanes 0..63 of the same column
+            if (sub >= 2) {
+              tmem_ld32(tt + c, dv);
+#pragma unroll
+              for (int v = 0; v < 32; ++v) xchg[v * 64 + (L - 64)] = dv[v];
+            }
+            epilogue_bar();
+            if (sub < 2) {
+              tmem_ld32(tt + c, dv);
+              const int col = w.nt * (BN / 2) + (int)rank * (BN / 4) + L;
+              if (col < ncols) {
+#pragma unroll
+                for (int v = 0; v < 32; ++v)
+                  if (c + v < w.tail)
+                    outb[(trow0 + c + v) * ncols + col] = bf16_bits(silu(dv[v]) * xchg[v * 64 + L]);
+              }
+            }
+            epilogue_bar();
+          } else {
+            tmem_ld32(tt + c, dv);
+            const int col = w.nt * BN + (int)rank * (BN / 2) + L;
+            if (col < ncols) {
+#pragma unroll
+              for (int v = 0; v < 32; ++v) {
+                if (c + v < w.tail) {
+                  const float sc = (!w.sh && p.row_scale) ? __ldg(p.row_scale + trow0 + c + v) : 1.0f;
+                  outb[(trow0 + c + v) * ncols + col] = bf16_bits(dv[v] * sc);
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(cluster_addr(&acc_empty[1], 0));
+      }
+      if (!pair_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err, peer_abort)) break;
+      ph_f ^= 1u << acc;
+      tc_fence_after();
+      const int m0 = w.mt * P_M + (int)rank * BM + sub * 32;   // group row of this warp's lane 0
+      const int m = m0 + lane;
+      const bool valid = m < w.rows;
+      const size_t orow = grow0 + m;
+      uint16_t* out = outb + orow * ncols;
+      const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+      if (m0 < w.rows) {                   // at least one valid row in this warp
+        if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+          for (int c = 0; c < BN / 2; c += 32) {
+            // output columns c .. c + 31 of the tile: gate in accumulator
+            // column gc (c < 64: c; else c + 64), up 64 columns further
+            const int gc = c < BN / 4 ? c : c + BN / 4;
+            float gv[32], uv[32];
+            tmem_ld32(tb + gc, gv);
+            tmem_ld32(tb + gc + BN / 4, uv);
+            const int col0 = w.nt * (BN / 2) + c;
+            if (valid) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                if (col0 + 8 * v < ncols) {
+                  uint4 pk;
+                  pk.x = pack_bf16(silu(gv[8 * v + 0]) * uv[8 * v + 0], silu(gv[8 * v + 1]) * uv[8 * v + 1]);
+                  pk.y = pack_bf16(silu(gv[8 * v + 2]) * uv[8 * v + 2], silu(gv[8 * v + 3]) * uv[8 * v + 3]);
+                  pk.z = pack_bf16(silu(gv[8 * v + 4]) * uv[8 * v + 4], silu(gv[8 * v + 5]) * uv[8 * v + 5]);
+                  pk.w = pack_bf16(silu(gv[8 * v + 6]) * uv[8 * v + 6], silu(gv[8 * v + 7]) * uv[8 * v + 7]);
+                  *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
+                }
+              }
+            }
+          }
+        } else {
+          const float scale = (!w.sh && p.row_scale && valid) ? __ldg(p.row_scale + orow) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float dv[32];
+            tmem_ld32(tb + c, dv);
+            const int col0 = w.nt * BN + c;
+            if (valid) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                if (col0 + 8 * v < ncols) {
+                  uint4 pk;
+                  pk.x = pack_bf16(dv[8 * v + 0] * scale, dv[8 * v + 1] * scale);
+                  pk.y = pack_bf16(dv[8 * v + 2] * scale, dv[8 * v + 3] * scale);
+                  pk.z = pack_bf16(dv[8 * v + 4] * scale, dv[8 * v + 5] * scale);
+                  pk.w = pack_bf16(dv[8 * v + 6] * scale, dv[8 * v + 7] * scale);
+                  *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(cluster_addr(&acc_empty[acc], 0));
+    }
+  }
+
+  // after a wait gave up, loads may still be landing in this CTA's shared
+  // memory (the odd CTA cannot observe its own: they complete on the even
+  // CTA's barrier); they finish within microseconds, so wait a millisecond
+  if (*abort_flag) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 1000000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();          // neither CTA leaves while the other may still signal it
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -896,8 +1397,123 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   return cudaGetLastError();
 }
 
+int tc_pair_min_rows() { return tc::kPairMinRows; }
+int tc_pair_rows() { return tc::P_M; }
+int tc_pair_merge_rows() { return tc::kPairMergeMax; }
+
+// Largest grid of CTA pairs that is resident at once (the pair kernel is
+// persistent: a pair that had to wait for another to finish would double the
+// time of its units).
+static int pair_grid(const void* kern, size_t smem) {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  cfg.blockDim = dim3(tc::NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  const int grid = 2 * std::min(n, num_sms() / 2);
+  if (dev < 64) cached[dev] = grid;
+  return grid;
+}
+
+static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st) {
+  using namespace tc;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaFuncSetAttribute(pair_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    cudaFuncSetAttribute(pair_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    attr_done[dev] = true;
+  }
+  const bool has_s = a.E_s > 0;
+  Params p{};
+  bool ok = true;
+  p.grp_rows = a.grp_rows;
+  p.grp_row0 = a.grp_row0;
+  p.G = a.E_r + a.E_s;
+  p.E_r = a.E_r;
+  p.err = a.err;
+  p.bk = BK;
+  const uint32_t half = BN / 2, quarter = BN / 4;
+  if (which == 0) {
+    // gate/up: A = permuted tokens (routed) or h (shared); B = 64 gate rows and
+    // the 64 up rows of the same columns per CTA
+    const uint64_t wr_r = (uint64_t)a.E_r * a.f_r, wr_s = has_s ? (uint64_t)a.E_s * a.f_s : wr_r;
+    const void* xs = has_s ? a.x_s : a.x_r;
+    const uint64_t xs_rows = has_s ? (uint64_t)a.T : (uint64_t)a.max_rows_r;
+    ok &= make_tmap(&p.a_r, a.x_r, (uint64_t)a.max_rows_r, a.d, BM);
+    ok &= make_tmap(&p.a_s, xs, xs_rows, a.d, BM);
+    ok &= make_tmap(&p.a32_r, a.x_r, (uint64_t)a.max_rows_r, a.d, A_SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, xs, xs_rows, a.d, A_SUB_ROWS);
+    ok &= make_tmap(&p.b0_r, a.wg_r, wr_r, a.d, quarter);
+    ok &= make_tmap(&p.b1_r, a.wu_r, wr_r, a.d, quarter);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wg_s : a.wg_r, wr_s, a.d, quarter);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wu_s : a.wu_r, wr_s, a.d, quarter);
+    p.prefix = a.pre_gu;
+    p.k_r = p.k_s = a.d;
+    p.wrows_r = a.f_r; p.wrows_s = a.f_s;
+    p.ncols_r = a.f_r; p.ncols_s = a.f_s;
+    p.out_r = (uint16_t*)a.act_r; p.out_s = (uint16_t*)a.act_s;
+    p.row_scale = nullptr;
+  } else {
+    // down: A = act (routed / shared); B = W_down, 128 of the tile's 256 rows per CTA
+    const uint64_t rows_s = has_s ? (uint64_t)a.E_s * a.T : (uint64_t)a.max_rows_r;
+    const int fs = has_s ? a.f_s : a.f_r;
+    const uint64_t wd_rows_s = (uint64_t)(has_s ? a.E_s : a.E_r) * a.d;
+    ok &= make_tmap(&p.a_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, BM);
+    ok &= make_tmap(&p.a_s, has_s ? a.act_s : a.act_r, rows_s, fs, BM);
+    ok &= make_tmap(&p.a32_r, a.act_r, (uint64_t)a.max_rows_r, a.f_r, A_SUB_ROWS);
+    ok &= make_tmap(&p.a32_s, has_s ? a.act_s : a.act_r, rows_s, fs, A_SUB_ROWS);
+    ok &= make_tmap(&p.b0_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, half);
+    ok &= make_tmap(&p.b1_r, a.wd_r, (uint64_t)a.E_r * a.d, a.f_r, half);
+    ok &= make_tmap(&p.b0_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, half);
+    ok &= make_tmap(&p.b1_s, has_s ? a.wd_s : a.wd_r, wd_rows_s, fs, half);
+    p.prefix = a.pre_dn;
+    p.k_r = a.f_r; p.k_s = a.f_s;
+    p.wrows_r = a.d; p.wrows_s = a.d;
+    p.ncols_r = a.d; p.ncols_s = a.d;
+    p.out_r = (uint16_t*)a.out_r; p.out_s = (uint16_t*)a.out_s;
+    p.row_scale = a.row_scale;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
+  auto kern = which == 0 ? pair_gemm_kernel<EPI_SWIGLU> : pair_gemm_kernel<EPI_SCALE>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pair_grid((const void*)kern, P_SMEM));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = P_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
   using namespace tc;
+  if (a.pair) return launch_ffn_pair(a, which, st);
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);

@@ -28,6 +28,9 @@ struct FfnArgs {
   float *as_r, *as_s;
   // training forward: U | V of every row ([rows, 2f] bf16) for the backward
   void *uv_r, *uv_s;
+  // 1: run both GEMMs on CTA pairs (tc_pair_rows()-row tiles, no merged
+  // tails; the group tables were built with that tile height)
+  int pair;
 };
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
@@ -136,6 +139,11 @@ void launch_bwd_gate_dh_de(const BwdRouteArgs& a, cudaStream_t st);   // dz, dh,
 
 int tc_bm();
 int tc_merge_rows();   // tails of <= this many rows share the unit of the tile before
+// CTA-pair GEMMs: rows per pair tile, and the mean routed rows per expert from
+// which bf16 inference layers use them
+int tc_pair_rows();
+int tc_pair_min_rows();
+int tc_pair_merge_rows();   // pair kernel: tails of <= this many rows share the unit before
 int tc_cols_gateup();
 int tc_cols_down();
 // which = 0: gate/up GEMM + SwiGLU epilogue; which = 1: down GEMM + gate scaling

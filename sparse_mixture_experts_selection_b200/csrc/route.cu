@@ -10,6 +10,7 @@
 //  "Mixture of Experts: Routing and Load Balancing": section 5 (capacity admits
 //   tokens in the order they appear).
 //  "GPUs, memory and failures": the bias card (update once per step).
+#include <algorithm>
 #include <cfloat>
 #include "common.cuh"
 #include "kernels.h"
@@ -480,6 +481,106 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ h, const int32_t* _
   }
 }
 
+// The same gather on the TMA engine's untiled bulk copies: one thread per CTA
+// streams whole rows h[perm_tok[r]] -> shared memory -> x_perm[r] through a
+// ring of n_buf row buffers (rows r = blockIdx.x + j * gridDim.x): n_buf -
+// kGatherStoresInFlight row loads and the shared-memory reads of up to
+// kGatherStoresInFlight row stores are in flight per CTA, and every write
+// leaves as whole lines.  Addresses and row_bytes are multiples of 16 (checked
+// by the launcher).  A row whose token index is out of range is neither read
+// nor written (MOE_DEVERR_INDEX); every wait is bounded.
+constexpr bool kGatherBulk = true;
+constexpr int kGatherRingBytes = 96 * 1024;   // ring bytes per CTA at most
+constexpr int kGatherMaxBuf = 16;
+constexpr int kGatherStoresInFlight = 2;
+
+__device__ __forceinline__ void bulk_load_row(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(sdst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_row(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(gdst), "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(32) gather_rows_bulk_kernel(
+    const uint8_t* __restrict__ h, const int32_t* __restrict__ perm_tok, const int* __restrict__ n_rows_ptr,
+    uint8_t* __restrict__ x_perm, int row_bytes, int n_buf, int max_my, int n_tok, int max_rows, int* err,
+    const float* __restrict__ s_src, float* __restrict__ s_dst) {
+  // n_buf row buffers, n_buf barriers, then the token of each of this CTA's rows
+  extern __shared__ __align__(128) uint8_t ring[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)n_buf * row_bytes);
+  int32_t* tok = reinterpret_cast<int32_t*>(full + n_buf);
+  __shared__ int abort_flag;
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    for (int b = 0; b < n_buf; ++b) mbar_init(&full[b], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();
+  pdl_trigger();
+  const int n = min(*n_rows_ptr, max_rows);
+  int my = n > (int)blockIdx.x ? (n - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  if (my > max_my) {                                   // cannot happen with the launcher's grid
+    if (lane == 0) set_device_error(err, MOE_DEVERR_INDEX);
+    my = max_my;
+  }
+  auto row_of_j = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
+  // all lanes fetch the tokens (and, for e4m3 rows, copy the row scales) so
+  // that the issuing lane never waits on a global load
+#pragma unroll 4
+  for (int j = lane; j < my; j += kWarp) {
+    const int r = row_of_j(j), t = perm_tok[r];
+    tok[j] = t;
+    if (s_src && (unsigned)t < (unsigned)n_tok) s_dst[r] = s_src[t];
+  }
+  __syncwarp();
+  if (lane != 0) return;
+  auto issue = [&](int j) {
+    const int b = j % n_buf;
+    const int t = tok[j];
+    if ((unsigned)t >= (unsigned)n_tok) {             // self-check: never read outside h
+      set_device_error(err, MOE_DEVERR_INDEX);
+      mbar_arrive(&full[b]);                           // completes the phase with no bytes
+      return;
+    }
+    mbar_arrive_expect_tx(&full[b], (uint32_t)row_bytes);
+    bulk_load_row(ring + (size_t)b * row_bytes, h + (size_t)t * row_bytes, (uint32_t)row_bytes, &full[b]);
+  };
+  // row j + ahead goes into the buffer of row j - kGatherStoresInFlight, whose
+  // store is the oldest of the kGatherStoresInFlight + 1 committed last
+  const int ahead = n_buf - kGatherStoresInFlight;
+  int issued = 0;
+  for (; issued < my && issued < ahead; ++issued) issue(issued);
+  for (int j = 0; j < my; ++j) {
+    const int b = j % n_buf;
+    if (!mbar_wait(&full[b], (uint32_t)(j / n_buf) & 1u, &abort_flag, err)) break;
+    if ((unsigned)tok[j] < (unsigned)n_tok) {
+      fence_proxy_async_smem();
+      bulk_store_row(x_perm + (size_t)row_of_j(j) * row_bytes, ring + (size_t)b * row_bytes, (uint32_t)row_bytes);
+    }
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");   // one group per row, even an empty one
+    if (issued < my) {
+      asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kGatherStoresInFlight) : "memory");
+      issue(issued++);
+    }
+  }
+  // after an abandoned wait, the loads still in flight (the last `ahead`
+  // issued at most) must land before the CTA exits
+  if (abort_flag) {
+    for (int j = max(0, issued - ahead); j < issued; ++j) {
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(&full[j % n_buf], (uint32_t)(j / n_buf) & 1u) &&
+             global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // dst[r] = src[map[r]] (map[r] < 0: a zero row) for r < n_rows; rows of
 // row_words 32-bit words, moved 16 bytes at a time when row_words % 4 == 0.
 __global__ void gather_map_kernel(const uint32_t* __restrict__ src, const int32_t* __restrict__ map,
@@ -852,11 +953,36 @@ void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
 void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
                    int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st,
                    const float* s_src, float* s_dst) {
+  const int row_bytes = d * elem_bytes;
+  const int n_buf = std::min(kGatherMaxBuf, kGatherRingBytes / std::max(row_bytes, 16));
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  sms = std::max(sms, 1);
+  const size_t ring = (size_t)n_buf * row_bytes + (size_t)n_buf * sizeof(uint64_t);
+  // as many CTAs per SM as their rings fit in 224 KB (at most 6)
+  const int per_sm = std::max(1, std::min(6, (224 * 1024) / (int)(ring + 1024 + 8 * 1024)));
+  const int blocks = std::min(std::max(max_rows, 1), per_sm * sms);
+  const int max_my = (std::max(max_rows, 1) + blocks - 1) / blocks;   // rows per CTA at most
+  const size_t smem = ring + (size_t)max_my * sizeof(int32_t);
+  if (kGatherBulk && n_buf >= kGatherStoresInFlight + 2 && row_bytes % 16 == 0 && max_my <= 2048 &&
+      ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(x_perm)) & 15) == 0) {
+    static bool attr_done[64] = {};
+    if (dev < 64 && !attr_done[dev]) {
+      cudaFuncSetAttribute(gather_rows_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kGatherRingBytes + kGatherMaxBuf * (int)sizeof(uint64_t) + 2048 * 4);
+      attr_done[dev] = true;
+    }
+    launch_pdl(gather_rows_bulk_kernel, dim3(blocks), dim3(kWarp), smem, st, (const uint8_t*)h, perm_tok,
+               n_rows_ptr, (uint8_t*)x_perm, row_bytes, n_buf, max_my, n_tok, max_rows, err, s_src, s_dst);
+    return;
+  }
   int vec = d * elem_bytes / 16;
   int warps = max_rows < 148 * 64 ? max_rows : 148 * 64;
   if (warps < 1) warps = 1;
-  int blocks = (warps * 32 + 255) / 256;
-  launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, (const uint4*)h, perm_tok, n_rows_ptr,
+  const int ldst_blocks = (warps * 32 + 255) / 256;
+  launch_pdl(gather_rows_kernel, dim3(ldst_blocks), dim3(256), 0, st, (const uint4*)h, perm_tok, n_rows_ptr,
              (uint4*)x_perm, vec, n_tok, max_rows, err, s_src, s_dst);
 }
 

@@ -251,6 +251,50 @@ def test_fullsize_every_tile_kind(name, weights_cache):
     print(f"{name}: every row of {n} experts ({R} rows) within the bar; kinds {sorted(set(kinds))}")
 
 
+# rows per expert reaching every CTA-pair tile kind (256-row tiles: the even
+# CTA holds rows 0..127, the odd one 128..255): two tiles + 188 rows (odd half
+# partial), one row, one row in the odd half, merged tails of 64 rows (the
+# largest) and of 48 rows after two tiles, a tile + 65 rows (the smallest
+# padded tail), a tile + 1 row (merged), an empty expert
+PAIR_ROWS = [700, 1, 129, 320, 560, 321, 257, 0]
+
+
+@pytest.mark.parametrize("name", ["mixtral_8x14336", "finegrained_64x1408"])
+def test_fullsize_pair_tiles(name, weights_cache):
+    """moe_expert_ffn on the CTA-pair GEMMs (>= 512 rows provisioned per
+    expert, as the layer provisions T*K/E_r at these shapes) at the workload's
+    full d and f; every output row of every expert element by element."""
+    w = mi.WORKLOADS[name]
+    n = min(len(PAIR_ROWS), w.E_r)
+    rows = np.array(PAIR_ROWS[:n])
+    offsets = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    R = int(offsets[-1])
+    max_rows = 512 * n
+    x = mi.gen_h(w, 0)[np.arange(R) % w.T]
+    gate = np.random.default_rng(4).uniform(0.05, 1.0, size=R).astype(np.float32)
+    Wd = _layer(w, weights_cache).W
+    cfg = moe.config_for(w)
+    ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n, w.d_ffn, max_rows))
+    xd = torch.zeros((max_rows, w.d_model), dtype=torch.bfloat16, device="cuda")
+    xd[:R] = to_dev(x, torch.bfloat16)
+    out = torch.empty((max_rows, w.d_model), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, n, w.d_ffn, max_rows, to_dev(offsets, torch.int32), xd,
+                       Wd["gate"][:n], Wd["up"][:n], Wd["down"][:n], to_dev(gate), out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    got = out[:R].float().cpu().numpy().astype(np.float64)
+    src = LazyHostWeights(w).source()
+    for ex in range(n):
+        r0, r1 = int(offsets[ex]), int(offsets[ex + 1])
+        if r0 == r1:
+            continue
+        want = gate[r0:r1, None].astype(np.float64) * mo.swiglu(x[r0:r1], src("gate", ex), src("up", ex),
+                                                                   src("down", ex))
+        diff = np.abs(got[r0:r1] - want) - 2.0 ** -8 * np.abs(want)
+        r = float(np.sqrt(np.mean(want ** 2)))
+        assert float(diff.max()) <= BF16_TOL * r, (ex, int(rows[ex]), float(diff.max()), r)
+
+
 def test_fullsize_shared_expert_slices(weights_cache):
     """The DeepSeek-V3 shared expert (all 4096 tokens, 32 full tiles at
     d = 7168) through moe_expert_ffn: the first, a middle and the last 128-row

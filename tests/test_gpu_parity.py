@@ -41,6 +41,10 @@ SMALL = {
                                              d_ffn_shared=384, n_groups=8, topk_groups=3),
     "decode_small": W["deepseek_v3_decode"].with_(T=24, d_model=320, E_r=64, d_ffn=128,
                                                   d_ffn_shared=128, topk_groups=4),
+    # >= 512 rows per routed expert: the GEMMs run on CTA pairs (256-row tiles)
+    "mixtral_pairs": W["mixtral_8x14336"].with_(T=2304, d_model=256, d_ffn=320),
+    "finegrained_pairs": W["finegrained_64x1408"].with_(T=1100, d_model=192, E_r=8, E_s=2, K=4,
+                                                        d_ffn=192, d_ffn_shared=136),
 }
 
 
@@ -239,6 +243,51 @@ def test_expert_ffn_entry(dtype):
     tol = BF16_TOL if dtype == "bf16" else F32_TOL
     err = np.max(np.abs(got[:R] - want) - eps * np.abs(want))
     assert err <= tol * np.sqrt(np.mean(want ** 2)), err
+    assert np.all(got[R:] == 7.0)                     # rows past offsets[n] untouched
+
+
+# Rows per expert reaching every CTA-pair tile kind (256-row tiles; the even
+# CTA holds rows 0..127 of a tile, the odd one rows 128..255): empty, one row,
+# a full even half with the odd half empty, one row in the odd half, one full
+# tile, merged tails of 1, 44 and 64 rows (the largest) after one tile and of
+# 48 rows after two, a tile + 65 rows (the smallest padded tail) and + 127
+# (even half partial, odd empty), two tiles + 188 rows (odd half partial).
+PAIR_ROWS = [0, 1, 128, 129, 256, 257, 300, 320, 560, 321, 383, 700]
+
+
+def test_expert_ffn_pair_tiles():
+    """moe_expert_ffn with >= 512 rows provisioned per expert (the CTA-pair
+    GEMMs), ragged gate/up and down column tiles (f = 200, d = 192): every
+    output row within the bar, rows past offsets[n] untouched."""
+    n_exp, d, f = len(PAIR_ROWS), 192, 200
+    rows = np.array(PAIR_ROWS, dtype=np.int64)
+    offsets = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    R = int(offsets[-1])
+    rng = np.random.default_rng(5)
+    rnd = lambda *s, sc=1.0: (rng.normal(size=s) * sc).astype(np.float32)
+    x = mi.round_bf16(rnd(R, d))
+    wg, wu = mi.round_bf16(rnd(n_exp, f, d, sc=d ** -0.5)), mi.round_bf16(rnd(n_exp, f, d, sc=d ** -0.5))
+    wd = mi.round_bf16(rnd(n_exp, d, f, sc=f ** -0.5))
+    scale = rng.uniform(0.1, 1, size=R).astype(np.float32)
+    cfg = moe.MoeConfig(T=R, d_model=d, E_r=n_exp, E_s=0, K=1, d_ffn=f, d_ffn_shared=0, score_fn=0,
+                        n_groups=1, topk_groups=1, group_topn=0, capacity_factor=0.0, dtype=1, add_residual=1)
+    max_rows = 512 * n_exp
+    ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n_exp, f, max_rows))
+    xd = torch.zeros((max_rows, d), dtype=torch.bfloat16, device="cuda")
+    xd[:R] = to_dev(x, torch.bfloat16)
+    out = torch.full((max_rows, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, n_exp, f, max_rows, to_dev(offsets, torch.int32), xd, to_dev(wg, torch.bfloat16),
+                       to_dev(wu, torch.bfloat16), to_dev(wd, torch.bfloat16), to_dev(scale), out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    got = out.float().cpu().numpy()
+    for g in range(n_exp):
+        a, b_ = offsets[g], offsets[g + 1]
+        if b_ == a:
+            continue
+        want = scale[a:b_, None] * mo.swiglu(x[a:b_], wg[g], wu[g], wd[g])
+        err = np.max(np.abs(got[a:b_] - want) - 2.0 ** -8 * np.abs(want))
+        assert err <= BF16_TOL * np.sqrt(np.mean(want ** 2)), (g, PAIR_ROWS[g], err)
     assert np.all(got[R:] == 7.0)                     # rows past offsets[n] untouched
 
 
