@@ -641,6 +641,16 @@ def kernel_records(w, kept_h, phase_ms, ms_per_step, moe):
     return gu, dn, layer, hbm, mma_peak, peak_kind
 
 
+def gemm_tile_rows(w, moe) -> int:
+    """Row-tile height of the layer's grouped GEMMs as the library chooses it:
+    256 on CTA pairs, 128 single-CTA tensor-core, the CUDA-core tile for fp32
+    (the layer provisions min(T*K, E_r * capacity) routed rows)."""
+    rows = w.T * w.K
+    if w.capacity_factor > 0:
+        rows = min(rows, w.E_r * int(math.floor(w.T * w.K * w.capacity_factor / w.E_r)))
+    return moe.moe_expert_ffn_tile_rows(moe.config_for(w), w.E_r, max(rows, 1))
+
+
 def launches_per_step(w) -> int:
     """Our kernels per layer step: [centroid split + router GEMM | CUDA-core
     logits], select, scan, scatter, row gather (e4m3: quantize h + gather),
@@ -685,6 +695,7 @@ def measure_extra(name, args, rank, world, dev, stream, moe, native, clocks):
     kept_h = run.kept.cpu().numpy()[warm:]
     counts_h = run.counts.cpu().numpy()[warm:]
     gu, dn, layer, _, _, _ = kernel_records(w, kept_h, phase_ms, ms, moe)
+    gu["tile_rows"] = dn["tile_rows"] = gemm_tile_rows(w, moe)
     rec = {"value": job_throughput(world, w.T, steps, elapsed_ms), "unit": "tokens/s", "ms_per_step": ms,
            "steps": steps, "warmup": warm, "dtype": {"bf16": "bf16", "bf16_e4m3": "e4m3"}.get(w.dtype, "f32"),
            "config": workload_config(w), "layer_roofline": layer, "gate_up_gemm": gu, "down_gemm": dn,
@@ -786,6 +797,7 @@ def run_ours(args, w, rank, world, local_rank):
         del pin_h, y_host, h_dev, y_dev
 
     gu, dn, layer, hbm, mma_peak, peak_kind = kernel_records(w, kept_h, phase_ms, ms_per_step, moe)
+    gu["tile_rows"] = dn["tile_rows"] = gemm_tile_rows(w, moe)
     # DRAM traffic per launch: the ncu capture's DRAM bytes over its implementation
     # bytes (profiles/traffic.json), scaled to this launch's implementation bytes
     traffic = None

@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 typedef enum {
   MOE_OK = 0,
@@ -192,6 +192,17 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* idx, const float* g
  * the tensor core's own summation order inside each 16-element step.
  */
 /* Workspace bytes moe_expert_ffn needs for these arguments (*bytes: HOST pointer). */
+/*
+ * Row-tile height of the GEMMs moe_expert_ffn runs for these arguments
+ * (*rows: HOST pointer): 256 when both GEMMs run on CTA pairs, 128 for the
+ * single-CTA tensor-core GEMMs, the CUDA-core tile for fp32.  moe_layer_forward
+ * makes the same choice with n_experts = E_r and max_rows = its routed rows
+ * (T*K, or E_r times the capacity), except that a training forward
+ * (cfg->train) keeps the single-CTA GEMMs.  Queries the current device's
+ * cluster occupancy once; launches nothing.
+ */
+moe_status moe_expert_ffn_tile_rows(const moe_config* cfg, int32_t n_experts, int32_t max_rows,
+                                    int32_t* rows);
 moe_status moe_expert_ffn_workspace_size(const moe_config* cfg, int32_t n_experts, int32_t d_ffn,
                                          int32_t max_rows, size_t* bytes);
 

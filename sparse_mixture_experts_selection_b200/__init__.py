@@ -23,7 +23,7 @@ __all__ = [
     "moe_layer_forward", "moe_get_device_error", "moe_clear_device_error", "alloc_workspace",
     "moe_router_stats", "moe_router_stats_workspace_size", "ROUTER_STATS", "moe_permute_noalloc",
     "moe_quantized_bytes", "moe_quantize_rows", "DTYPE_BF16_E4M3", "moe_layer_backward", "moe_gather_rows",
-    "moe_set_phase_events", "moe_selftest_bounded_wait", "moe_ep_plan",
+    "moe_set_phase_events", "moe_selftest_bounded_wait", "moe_ep_plan", "moe_expert_ffn_tile_rows",
     "SCORE_SIGMOID", "SCORE_SOFTMAX", "DTYPE_F32", "DTYPE_BF16",
 ]
 
@@ -61,6 +61,7 @@ SIGNATURES = {
     "moe_last_error_detail": (ctypes.c_char_p, []),
     "moe_workspace_size": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_expert_ffn_workspace_size": (ctypes.c_int, [_P, _I32, _I32, _I32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_expert_ffn_tile_rows": (ctypes.c_int, [_P, _I32, _I32, ctypes.POINTER(ctypes.c_int32)]),
     "moe_route": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -147,6 +148,14 @@ def moe_workspace_size(cfg: MoeConfig) -> int:
 def moe_expert_ffn_workspace_size(cfg: MoeConfig, n_experts: int, d_ffn: int, max_rows: int) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().moe_expert_ffn_workspace_size(ctypes.byref(cfg), n_experts, d_ffn, max_rows, ctypes.byref(n)))
+    return n.value
+
+
+def moe_expert_ffn_tile_rows(cfg: MoeConfig, n_experts: int, max_rows: int) -> int:
+    """Row-tile height of the GEMMs moe_expert_ffn runs for these arguments:
+    256 on CTA pairs, 128 single-CTA tensor-core, the CUDA-core tile for fp32."""
+    n = ctypes.c_int32(0)
+    _check(lib().moe_expert_ffn_tile_rows(ctypes.byref(cfg), n_experts, max_rows, ctypes.byref(n)))
     return n.value
 
 

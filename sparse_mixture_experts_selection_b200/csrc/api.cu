@@ -224,17 +224,21 @@ void mark_phase(int i, cudaStream_t st) {
   if (i < g_n_phase_events && g_phase_events[i]) cudaEventRecord(g_phase_events[i], st);
 }
 
+// bf16 grouped FFNs whose experts average many rows (the rows the caller
+// provisions per routed expert: T*K/E_r in a dropless layer) run their GEMMs
+// on CTA pairs (256-row tiles), unless they keep U | V for a backward.
+static bool ffn_on_pairs(const moe_config& c, bool keeps_uv, int n_experts, int64_t max_rows) {
+  return use_tensor_cores(c.dtype) && !is_q8(c.dtype) && !keeps_uv && n_experts > 0 &&
+         max_rows >= (int64_t)moe::tc_pair_min_rows() * n_experts && moe::tc_pair_available();
+}
+
 // Group tables + both GEMMs of the grouped FFN (phase marks 3 and 4 after the
 // group tables and the gate/up GEMM when phase_base >= 0).
 moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int max_rows,
                    cudaStream_t st, int phase_base = -1) {
   const bool tc = use_tensor_cores(c.dtype);
-  // bf16 inference layers whose experts average many rows (the rows the
-  // caller provisions per routed expert: T*K/E_r in a dropless layer) run
-  // their GEMMs on CTA pairs (256-row tiles); the group tables follow that
-  // tile height
-  a.pair = tc && !a.q8 && a.uv_r == nullptr && a.E_r > 0 &&
-           (int64_t)max_rows >= (int64_t)moe::tc_pair_min_rows() * a.E_r;
+  // the group tables follow the tile height of the GEMMs that will run
+  a.pair = ffn_on_pairs(c, a.uv_r != nullptr, a.E_r, max_rows);
   const int bm = a.pair ? moe::tc_pair_rows() : tc ? moe::tc_bm() : moe::simt_bm();
   const int bn_gu = tc ? moe::tc_cols_gateup() : moe::simt_bn();
   const int bn_dn = tc ? moe::tc_cols_down() : moe::simt_bn();
@@ -269,6 +273,19 @@ moe_status run_ffn(const moe_config& c, moe::FfnArgs& a, const int* offsets, int
 extern "C" {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status moe_expert_ffn_tile_rows(const moe_config* cfg, int32_t n_experts, int32_t max_rows, int32_t* rows) {
+  MOE_CHECK(validate(cfg));
+  if (!rows) return fail(MOE_ERR_INVALID_ARG, "rows is NULL");
+  if (n_experts < 1 || max_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_experts=%d max_rows=%d", n_experts, max_rows);
+  const moe_config& c = *cfg;
+  if (!use_tensor_cores(c.dtype)) {
+    *rows = moe::simt_bm();
+    return MOE_OK;
+  }
+  *rows = ffn_on_pairs(c, false, n_experts, max_rows) ? moe::tc_pair_rows() : moe::tc_bm();
+  return MOE_OK;
+}
 
 const char* moe_status_string(moe_status s) {
   switch (s) {

@@ -1430,7 +1430,7 @@ static int pair_grid(const void* kern, size_t smem) {
   return grid;
 }
 
-static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st) {
+static void pair_attributes() {
   using namespace tc;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -1440,6 +1440,20 @@ static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st)
     cudaFuncSetAttribute(pair_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
     attr_done[dev] = true;
   }
+}
+
+// The pair kernels are worth launching only if the device co-schedules pairs
+// on at least three quarters of its SMs (a B200 holds 74 two-CTA clusters of
+// this kernel at once).
+bool tc_pair_available() {
+  pair_attributes();
+  const int g = pair_grid((const void*)tc::pair_gemm_kernel<tc::EPI_SWIGLU>, tc::P_SMEM);
+  return g >= (3 * num_sms()) / 4;
+}
+
+static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st) {
+  using namespace tc;
+  pair_attributes();
   const bool has_s = a.E_s > 0;
   Params p{};
   bool ok = true;

@@ -144,6 +144,7 @@ int tc_merge_rows();   // tails of <= this many rows share the unit of the tile 
 int tc_pair_rows();
 int tc_pair_min_rows();
 int tc_pair_merge_rows();   // pair kernel: tails of <= this many rows share the unit before
+bool tc_pair_available();   // the device co-schedules enough CTA pairs of the pair kernel
 int tc_cols_gateup();
 int tc_cols_down();
 // which = 0: gate/up GEMM + SwiGLU epilogue; which = 1: down GEMM + gate scaling

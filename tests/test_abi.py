@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     for s in syms:
         assert hasattr(L, s), s
     assert set(syms) == set(moe.SIGNATURES), set(syms) ^ set(moe.SIGNATURES)
-    assert L.moe_abi_version() == 3
+    assert L.moe_abi_version() == 4
     assert moe.lib().moe_status_string(3) == b"MOE_ERR_WORKSPACE"
 
 
@@ -76,6 +76,18 @@ def test_group_constraints():
     # topk_groups * group size < K
     c = cfg_of("deepseek_v3", topk_groups=1, K=33)
     assert L.moe_workspace_size(ctypes.byref(c), ctypes.byref(n)) in (1, 2)
+
+
+def test_expert_ffn_tile_rows_validation_and_fp32():
+    """The tile query validates on the host; an fp32 layer answers with the
+    CUDA-core tile without touching the device."""
+    L = moe.lib()
+    c = cfg_of("toy_fp32")
+    n = ctypes.c_int32(-1)
+    assert L.moe_expert_ffn_tile_rows(ctypes.byref(c), 8, 1024, None) == 1
+    assert L.moe_expert_ffn_tile_rows(ctypes.byref(c), 0, 1024, ctypes.byref(n)) == 1
+    assert L.moe_expert_ffn_tile_rows(ctypes.byref(c), 8, -1, ctypes.byref(n)) == 1
+    assert moe.moe_expert_ffn_tile_rows(c, 8, 4096) == 32
 
 
 def test_bf16_small_dims_unsupported():

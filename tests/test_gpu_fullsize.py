@@ -231,6 +231,7 @@ def test_fullsize_every_tile_kind(name, weights_cache):
     gate = np.random.default_rng(3).uniform(0.05, 1.0, size=R).astype(np.float32)
     Wd = _layer(w, weights_cache).W
     cfg = moe.config_for(w)
+    assert moe.moe_expert_ffn_tile_rows(cfg, n, R) == BM                  # the single-CTA tiles
     ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n, w.d_ffn, R))
     out = torch.empty((R, w.d_model), dtype=torch.bfloat16, device="cuda")
     moe.moe_expert_ffn(cfg, n, w.d_ffn, R, to_dev(offsets, torch.int32), to_dev(x, torch.bfloat16),
@@ -270,6 +271,7 @@ def test_fullsize_pair_tiles(name, weights_cache):
     offsets = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
     R = int(offsets[-1])
     max_rows = 512 * n
+    assert moe.moe_expert_ffn_tile_rows(moe.config_for(w), n, max_rows) == 256     # CTA pairs
     x = mi.gen_h(w, 0)[np.arange(R) % w.T]
     gate = np.random.default_rng(4).uniform(0.05, 1.0, size=R).astype(np.float32)
     Wd = _layer(w, weights_cache).W

@@ -223,6 +223,7 @@ def test_expert_ffn_entry(dtype):
                         n_groups=1, topk_groups=1, group_topn=0, capacity_factor=0.0,
                         dtype=1 if dtype == "bf16" else 0, add_residual=1)
     max_rows = R + 3
+    assert moe.moe_expert_ffn_tile_rows(cfg, n_exp, max_rows) == (128 if dtype == "bf16" else 32)
     ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n_exp, f, max_rows))
     xd = torch.zeros((max_rows, d), dtype=dt, device="cuda")
     xd[:R] = to_dev(x, dt)
@@ -272,6 +273,7 @@ def test_expert_ffn_pair_tiles():
     cfg = moe.MoeConfig(T=R, d_model=d, E_r=n_exp, E_s=0, K=1, d_ffn=f, d_ffn_shared=0, score_fn=0,
                         n_groups=1, topk_groups=1, group_topn=0, capacity_factor=0.0, dtype=1, add_residual=1)
     max_rows = 512 * n_exp
+    assert moe.moe_expert_ffn_tile_rows(cfg, n_exp, max_rows) == 256        # CTA pairs
     ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n_exp, f, max_rows))
     xd = torch.zeros((max_rows, d), dtype=torch.bfloat16, device="cuda")
     xd[:R] = to_dev(x, torch.bfloat16)
@@ -340,6 +342,17 @@ def test_bias_update_entry_bit_exact():
 # ---------------------------------------------------------------------------
 # the whole layer
 # ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_layer_gemm_tile_choice(name):
+    """bf16 layers provisioning >= 512 rows per routed expert (T*K/E_r) take
+    the CTA-pair GEMMs, the others the single-CTA ones; fp32 the CUDA cores."""
+    w = SMALL[name]
+    want = 32 if w.dtype == "f32" else (256 if w.T * w.K >= 512 * w.E_r else 128)
+    assert moe.moe_expert_ffn_tile_rows(moe.config_for(w), w.E_r, w.T * w.K) == want
+    if name.endswith("_pairs"):
+        assert want == 256
+
 
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_layer_fed_scores(name):
