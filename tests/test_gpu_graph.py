@@ -1,9 +1,10 @@
 """The layer forward captured in a CUDA graph.  moe_layer_forward only
 enqueues work on the caller's stream (kernels launched with programmatic
-dependent launch, a memset, no host synchronisation, no allocation), so a
-caller can capture a whole step -- routing, dispatch, both grouped GEMMs,
-combine and the bias step -- once and replay it.  Replays must match eager
-calls bit for bit, step after step, including the carried bias."""
+dependent launch, cluster launches for the CTA-pair GEMMs, a memset, no host
+synchronisation, no allocation), so a caller can capture a whole step --
+routing, dispatch, both grouped GEMMs, combine and the bias step -- once and
+replay it.  Replays must match eager calls bit for bit, step after step,
+including the carried bias."""
 import numpy as np
 import pytest
 import torch
@@ -18,12 +19,18 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 
-@pytest.mark.parametrize("name", ["deepseek_v3", "mixtral_8x14336"])
+@pytest.mark.parametrize("name", ["deepseek_v3", "mixtral_8x14336", "mixtral_8x14336_pairs"])
 def test_layer_forward_graph_replay_matches_eager(name):
-    w = mi.WORKLOADS[name].with_(T=256, d_model=256, d_ffn=256, d_ffn_shared=128,
-                                  E_r=min(mi.WORKLOADS[name].E_r, 32))
+    base = name.replace("_pairs", "")
+    w = mi.WORKLOADS[base].with_(T=256, d_model=256, d_ffn=256, d_ffn_shared=128,
+                                  E_r=min(mi.WORKLOADS[base].E_r, 32))
     if w.n_groups > 1:
         w = w.with_(n_groups=8, topk_groups=4)
+    if name.endswith("_pairs"):
+        # >= 512 rows per expert: the CTA-pair GEMMs (cluster launches), whose
+        # units are claimed dynamically -- replays must still match bit for bit
+        w = w.with_(T=2304)
+        assert moe.moe_expert_ffn_tile_rows(moe.config_for(w), w.E_r, w.T * w.K) == 256
     Wd = HostWeights(w).device()
     e = to_dev(mi.gen_centroids(w))
     b0 = mi.gen_bias(w)
