@@ -92,7 +92,8 @@ enum {
 enum {
   MOE_DEVERR_NONE = 0,
   MOE_DEVERR_WAIT_TIMEOUT = 1,   /* a pipeline barrier wait gave up (bounded spin) */
-  MOE_DEVERR_INDEX = 2           /* an expert index outside [0, E_r) was met       */
+  MOE_DEVERR_INDEX = 2,          /* an expert index outside [0, E_r) was met       */
+  MOE_DEVERR_RANGE = 3           /* a layer's fp16 slot row saturated (|v| > 65504) */
 };
 
 typedef struct {
@@ -247,6 +248,10 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float g
  *   s_in: optional fed scores [T, E_r] (skips the affinity; e may then be NULL).
  * With update_bias, the routing of THIS call uses the incoming b and the step
  * is applied afterwards (the bias is carried to the next step).
+ * Inside the workspace a bf16 layer keeps the gate-weighted expert rows and
+ * the shared experts' outputs in fp16 (11 significant bits, 2 bytes) until the
+ * combine adds them in fp32: a value beyond +-65504 saturates and sets
+ * MOE_DEVERR_RANGE.  The standalone moe_expert_ffn / moe_combine keep cfg->dtype.
  */
 moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* e, float* b,
                              const void* w_gate, const void* w_up, const void* w_down,

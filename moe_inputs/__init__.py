@@ -11,12 +11,22 @@ Generator (counter-based, so any slice of any tensor can be regenerated alone):
   pseudorandom number generators", OOPSLA 2014) applied to a Weyl sequence:
   draw n of stream (seed, tensor_id) is ``mix(key + (n + 1) * GOLDEN)`` with
   ``key = mix(mix(seed) + tensor_id * GOLDEN)`` (all mod 2**64).
-* Normal variates: the four 16-bit fields of one draw are summed (an
-  Irwin-Hall sum of four discrete uniforms), centred, and scaled by
-  sqrt(3)/65536 so the variance is 1 (to within 2**-32).  Only integer
-  arithmetic and one IEEE double multiply are involved, so the CUDA twin in
-  ``gen.cu`` reproduces every value bit for bit.  The support is bounded at
-  +-3.46 sigma, which is immaterial for these workloads.
+* Normal variates: the Box-Muller transform (Box & Muller, "A note on the
+  generation of random normal deviates", Ann. Math. Statist. 1958) of the two
+  32-bit halves of one draw: u1 = (hi + 1/2) 2**-32 in (0, 1), u2 = lo 2**-32,
+  z = sqrt(-2 ln u1) cos(2 pi u2), times sigma.  ln and cos are evaluated by
+  fixed series in plain IEEE double operations, each rounded on its own (no
+  library call, no fused multiply-add), so that the C and CUDA twins in
+  ``gen.cu`` reproduce every value bit for bit:
+  - ln x for x = hi + 1/2: x = m 2**e exactly with m in [sqrt(1/2), sqrt(2)),
+    ln m = 2 atanh(s) = 2 s (1 + s^2/3 + s^4/5 + ... + s^20/21) with
+    s = (m - 1)/(m + 1), |s| <= 0.172 (the truncated terms are below 2**-60
+    relative), and ln u1 = ln m + (e - 32) ln 2;
+  - cos(2 pi u2): the quadrant and the position in it come exactly from the
+    integer lo; the angle is folded into [0, pi/4] (theta = g pi / 2**31 with
+    g <= 2**29) and cos theta, sin theta are Taylor series to the theta^20 and
+    theta^21 terms (the remainders are below 2**-70).
+  The tails reach +-6.76 sigma (u1 >= 2**-33).
 * Uniform variates: the top 53 bits of one draw, mapped to [lo, hi) in double.
 * Rounding: double -> float32 round-to-nearest-even, then (bf16 tensors)
   float32 -> bf16 round-to-nearest-even.
@@ -37,8 +47,25 @@ MASK64 = (1 << 64) - 1
 GOLDEN = 0x9E3779B97F4A7C15
 _M1 = 0xBF58476D1CE4E5B9
 _M2 = 0x94D049BB133111EB
-SQRT3_OVER_65536 = math.sqrt(3.0) / 65536.0
-IRWIN_HALL_CENTRE = 131070  # 4 * 32767.5
+
+# Constants of the normal variates as exact double bit patterns (the same hex
+# literals stand in gen.cu): ln 2, sqrt(1/2), pi / 2**31, and the series
+# coefficients 1/(2k+1), (-1)^k/(2k)!, (-1)^k/(2k+1)! for k = 0..10.
+_LN2 = float.fromhex("0x1.62e42fefa39efp-1")
+_SQRT_HALF = float.fromhex("0x1.6a09e667f3bcdp-1")
+_PI_OVER_2_31 = float.fromhex("0x1.921fb54442d18p-30")
+_LN_C = [float.fromhex(h) for h in (
+    "0x1.0000000000000p+0", "0x1.5555555555555p-2", "0x1.999999999999ap-3", "0x1.2492492492492p-3",
+    "0x1.c71c71c71c71cp-4", "0x1.745d1745d1746p-4", "0x1.3b13b13b13b14p-4", "0x1.1111111111111p-4",
+    "0x1.e1e1e1e1e1e1ep-5", "0x1.af286bca1af28p-5", "0x1.8618618618618p-5")]
+_COS_C = [float.fromhex(h) for h in (
+    "0x1.0000000000000p+0", "-0x1.0000000000000p-1", "0x1.5555555555555p-5", "-0x1.6c16c16c16c17p-10",
+    "0x1.a01a01a01a01ap-16", "-0x1.27e4fb7789f5cp-22", "0x1.1eed8eff8d898p-29", "-0x1.93974a8c07c9dp-37",
+    "0x1.ae7f3e733b81fp-45", "-0x1.6827863b97d97p-53", "0x1.e542ba4020225p-62")]
+_SIN_C = [float.fromhex(h) for h in (
+    "0x1.0000000000000p+0", "-0x1.5555555555555p-3", "0x1.1111111111111p-7", "-0x1.a01a01a01a01ap-13",
+    "0x1.71de3a556c734p-19", "-0x1.ae64567f544e4p-26", "0x1.6124613a86d09p-33", "-0x1.ae7f3e733b81fp-41",
+    "0x1.952c77030ad4ap-49", "-0x1.2f49b46814157p-57", "0x1.71b8ef6dcf572p-66")]
 
 # tensor ids of one workload's streams (the step index is folded in for h)
 TID_H, TID_E, TID_B, TID_WG, TID_WU, TID_WD, TID_WSG, TID_WSU, TID_WSD = range(1, 10)
@@ -81,21 +108,53 @@ def raw_draws(seed: int, tensor_id: int, start: int, count: int) -> np.ndarray:
     return out
 
 
-def normal_scale(sigma: float) -> float:
-    return float(sigma) * SQRT3_OVER_65536
+def _horner(coeffs, w: np.ndarray) -> np.ndarray:
+    """c0 + w (c1 + w (c2 + ...)), one rounded multiply and one rounded add per step."""
+    p = np.full_like(w, coeffs[-1])
+    for c in reversed(coeffs[:-1]):
+        p = p * w
+        p = p + c
+    return p
+
+
+def ln_half_int(hi: np.ndarray) -> np.ndarray:
+    """ln(hi + 1/2) - 32 ln 2 = ln(u1) for 32-bit integers hi (see module docstring)."""
+    x = hi.astype(np.float64) + 0.5
+    m, e = np.frexp(x)                         # x = m 2**e, m in [1/2, 1), exact
+    low = m < _SQRT_HALF
+    m = np.where(low, m * 2.0, m)
+    e = np.where(low, e - 1, e)
+    s = (m - 1.0) / (m + 1.0)
+    p = _horner(_LN_C, s * s)
+    return (s * 2.0) * p + (e - 32).astype(np.float64) * _LN2
+
+
+def cos_2pi_frac(lo: np.ndarray) -> np.ndarray:
+    """cos(2 pi lo / 2**32) for 32-bit integers lo (see module docstring)."""
+    lo = lo.astype(np.int64)
+    q = lo >> 30                               # quadrant
+    f = lo & ((1 << 30) - 1)                   # position in it, angle f pi / 2**31
+    fold = f >= (1 << 29)
+    g = np.where(fold, (1 << 30) - f, f).astype(np.float64)
+    th = g * _PI_OVER_2_31                     # in [0, pi/4]
+    w = th * th
+    c = _horner(_COS_C, w)
+    sn = th * _horner(_SIN_C, w)
+    ca = np.where(fold, sn, c)                 # cos and sin of the angle within the quadrant
+    sa = np.where(fold, c, sn)
+    return np.select([q == 0, q == 1, q == 2], [ca, -sa, -ca], sa)
 
 
 def normal_f32(seed: int, tensor_id: int, start: int, count: int, sigma: float) -> np.ndarray:
-    """float32 N(0, sigma^2) stand-ins (see module docstring)."""
-    scale = normal_scale(sigma)
+    """float32 N(0, sigma^2) draws (Box-Muller; see module docstring)."""
     out = np.empty(count, dtype=np.float32)
+    sig = float(sigma)
     for c0 in range(0, count, _CHUNK):
         c1 = min(count, c0 + _CHUNK)
         r = raw_draws(seed, tensor_id, start + c0, c1 - c0)
-        s = (r & np.uint64(0xFFFF)) + ((r >> np.uint64(16)) & np.uint64(0xFFFF)) \
-            + ((r >> np.uint64(32)) & np.uint64(0xFFFF)) + (r >> np.uint64(48))
-        cen = s.astype(np.int64) - IRWIN_HALL_CENTRE
-        out[c0:c1] = (cen.astype(np.float64) * scale).astype(np.float32)
+        rad = np.sqrt(ln_half_int(r >> np.uint64(32)) * -2.0)
+        z = rad * cos_2pi_frac(r & np.uint64(0xFFFFFFFF))
+        out[c0:c1] = (z * sig).astype(np.float32)
     return out
 
 

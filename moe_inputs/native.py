@@ -8,7 +8,7 @@ import subprocess
 
 import numpy as np
 
-from . import normal_scale, weight_spec, h_tensor_id, TID_E, Workload
+from . import weight_spec, h_tensor_id, TID_E, Workload
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoegen.so")
@@ -47,7 +47,7 @@ def lib():
 
 def fill_device(ptr: int, count: int, bf16: bool, seed: int, tensor_id: int, start: int,
                 sigma: float = 1.0, uniform=None, stream: int = 0) -> None:
-    kind, p0, p1 = (0, normal_scale(sigma), 0.0) if uniform is None else \
+    kind, p0, p1 = (0, float(sigma), 0.0) if uniform is None else \
         (1, float(uniform[0]), float(uniform[1]) - float(uniform[0]))
     rc = lib().moe_gen_fill_device(ctypes.c_void_p(ptr), count, int(bf16), kind, seed, tensor_id,
                                    start, p0, p1, ctypes.c_void_p(stream))
@@ -58,7 +58,7 @@ def fill_device(ptr: int, count: int, bf16: bool, seed: int, tensor_id: int, sta
 def fill_host(count: int, bf16: bool, seed: int, tensor_id: int, start: int, sigma: float = 1.0,
               uniform=None, threads: int = 0) -> np.ndarray:
     """Host twin: returns uint16 bf16 bits (bf16=True) or float32."""
-    kind, p0, p1 = (0, normal_scale(sigma), 0.0) if uniform is None else \
+    kind, p0, p1 = (0, float(sigma), 0.0) if uniform is None else \
         (1, float(uniform[0]), float(uniform[1]) - float(uniform[0]))
     out = np.empty(count, dtype=np.uint16 if bf16 else np.float32)
     lib().moe_gen_fill_host(out.ctypes.data_as(ctypes.c_void_p), count, int(bf16), kind, seed,

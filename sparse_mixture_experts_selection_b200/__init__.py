@@ -29,7 +29,7 @@ __all__ = [
 
 SCORE_SIGMOID, SCORE_SOFTMAX = 0, 1
 DTYPE_F32, DTYPE_BF16, DTYPE_BF16_E4M3 = 0, 1, 2
-DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_INDEX = 0, 1, 2
+DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_INDEX, DEVERR_RANGE = 0, 1, 2, 3
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
 

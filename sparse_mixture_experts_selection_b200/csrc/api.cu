@@ -526,11 +526,14 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* h, const float* 
     a.actq_r = at<void>(ws, L.actq_r); a.actq_s = c.E_s ? at<void>(ws, L.actq_s) : a.actq_r;
     a.as_r = at<float>(ws, L.as_r); a.as_s = c.E_s ? at<float>(ws, L.as_s) : a.as_r;
   }
+  // the slot and shared rows stay inside the workspace: fp16 for a bf16
+  // layer (three more significant bits than bf16 in the same bytes)
+  a.out_f16 = use_tensor_cores(c.dtype) ? 1 : 0;
   MOE_CHECK(run_ffn(c, a, offsets, (int)L.R, st, 3));
   mark_phase(5, st);
   // a8: fixed-order combine with the residual
   moe::launch_combine(h, a.out_r, c.E_s ? a.out_s : nullptr, row_of, y, c.T, c.d_model, c.K, c.E_s,
-                      c.add_residual, act_dtype(c.dtype), (int)L.R, st);
+                      c.add_residual, act_dtype(c.dtype), (int)L.R, st, a.out_f16);
   mark_phase(6, st);
   // a9: the bias step, after this batch's loads are counted
   if (update_bias || max_vio_out)
@@ -580,6 +583,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* h, const float*
   ra.dO = at<uint16_t>(ws, L.dO); ra.dh = static_cast<uint16_t*>(dh);
   ra.dg_row = at<float>(ws, L.dg_row); ra.dz = at<float>(ws, L.dz); ra.de = de;
   ra.err = err;
+  ra.slot_f16 = 1;                     // the forward (train = 1, bf16) wrote fp16 slot rows
   if (c.score_fn == MOE_SCORE_SIGMOID) {
     // the forward's per-chunk histogram, scanned without a capacity and
     // scattered stably: every selected pair by expert, tokens ascending

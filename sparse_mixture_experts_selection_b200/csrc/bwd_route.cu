@@ -14,6 +14,17 @@
 namespace moe {
 namespace {
 
+// eight fp16 values of a 16-byte vector (the layer's slot rows)
+__device__ __forceinline__ void unpack8_f16(uint4 q, float* v) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
 __device__ __forceinline__ void unpack8(uint4 q, float* v) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -28,7 +39,9 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// One warp per permuted row: dO = g * dy (bf16) and dL/dg = <dy, slot> / g.
+// One warp per permuted row: dO = g * dy (bf16) and dL/dg = <dy, slot> / g
+// (slot rows in fp16 when SLOT_F16, the layer's own, else bf16).
+template <bool SLOT_F16>
 __global__ void __launch_bounds__(256)
 bwd_rows_kernel(const uint16_t* __restrict__ dy, const int32_t* __restrict__ perm_tok,
                 const float* __restrict__ row_gate, const uint16_t* __restrict__ slot,
@@ -65,7 +78,7 @@ bwd_rows_kernel(const uint16_t* __restrict__ dy, const int32_t* __restrict__ per
         if (c >= d) break;
         float a[8], b[8];
         unpack8(qa[u], a);
-        unpack8(qb[u], b);
+        if (SLOT_F16) unpack8_f16(qb[u], b); else unpack8(qb[u], b);
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc = fmaf(a[i], b[i], acc);
         *reinterpret_cast<uint4*>(out + c) = make_uint4(pack2(g * a[0], g * a[1]), pack2(g * a[2], g * a[3]),
@@ -256,7 +269,8 @@ void launch_zero_tail_rows(void* buf, const int* n_rows_ptr, int max_rows, int c
 
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st) {
   const int warps = a.max_rows < 148 * 64 ? (a.max_rows > 0 ? a.max_rows : 1) : 148 * 64;
-  bwd_rows_kernel<<<(warps * kWarp + 255) / 256, 256, 0, st>>>(
+  auto kern = a.slot_f16 ? bwd_rows_kernel<true> : bwd_rows_kernel<false>;
+  kern<<<(warps * kWarp + 255) / 256, 256, 0, st>>>(
       a.dy, a.perm_tok, a.row_gate, a.slot, a.n_rows_ptr, a.max_rows, a.T, a.d, a.dO, a.dg_row, a.err);
 }
 

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "../../include/moe.h"
 
@@ -26,6 +27,27 @@ template <> __device__ __forceinline__ float to_f32<bf16>(bf16 v) { return __bfl
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+// The layer's slot rows (gate-weighted expert outputs) and shared-expert rows
+// are kept in fp16: 11 significant bits where bf16 has 8, in the same 2 bytes.
+// Values beyond the largest finite fp16 saturate to it (NaN stays NaN) and the
+// caller reports MOE_DEVERR_RANGE.
+constexpr float kF16Max = 65504.0f;
+__device__ __forceinline__ float f16_saturate(float v, bool& hit) {
+  if (fabsf(v) > kF16Max) {
+    hit = true;
+    return copysignf(kF16Max, v);
+  }
+  return v;
+}
+__device__ __forceinline__ uint32_t pack_f16_sat(float a, float b, bool& hit) {
+  __half2 v = __floats2half2_rn(f16_saturate(a, hit), f16_saturate(b, hit));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint16_t f16_bits_sat(float a, bool& hit) {
+  return __half_as_ushort(__float2half_rn(f16_saturate(a, hit)));
+}
 
 // ---------------------------------------------------------------------------
 // device error word (first 4 bytes of every workspace): the first error wins

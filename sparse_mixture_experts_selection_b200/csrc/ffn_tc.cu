@@ -116,6 +116,8 @@ struct Params {
   // [rows, 2f] bf16 (U in columns 0..f-1, V in f..2f-1), for the backward
   uint16_t* uv_r;
   uint16_t* uv_s;
+  // EPI_SCALE: 1 = outputs in fp16 (saturating, MOE_DEVERR_RANGE), else bf16
+  int out_f16;
 };
 
 constexpr int UNIT_RING = 4;     // units handed from the producer to the MMA / epilogue warps
@@ -232,6 +234,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Down-GEMM outputs: bf16, or saturating fp16 for a layer's own slot rows
+// (hit records a saturation, reported as MOE_DEVERR_RANGE).
+__device__ __forceinline__ uint32_t pack_out(int f16, float a, float b, bool& hit) {
+  return f16 ? pack_f16_sat(a, b, hit) : pack_bf16(a, b);
+}
+__device__ __forceinline__ uint16_t bits_out(int f16, float a, bool& hit) {
+  return f16 ? f16_bits_sat(a, hit) : bf16_bits(a);
+}
+
 // Tensor-map coordinates of the A and B tiles of k-block i of unit w.
 template <int EPI>
 struct TileCoords {
@@ -282,6 +293,7 @@ __device__ __noinline__ void epilogue_transposed(const Params& p, bool sh, uint1
     if (EPI == EPI_SWIGLU) cB = __ldg(wsB + colA);
   }
   if (EPI == EPI_SCALE && xs && colB < ncols) cB = __ldg(wsA + colB);
+  bool hit = false;
 #pragma unroll 1
   for (int c = 0; c < n16; c += 32) {
     float dv0[32], dv1[32];
@@ -304,12 +316,13 @@ __device__ __noinline__ void epilogue_transposed(const Params& p, bool sh, uint1
           }
         } else {
           const float sc = (!sh && p.row_scale) ? __ldg(p.row_scale + row0 + t) : 1.0f;
-          if (colA < ncols) orow_p[colA] = bf16_bits(dv0[v] * (rs * cA) * sc);
-          if (colB < ncols) orow_p[colB] = bf16_bits(dv1[v] * (rs * cB) * sc);
+          if (colA < ncols) orow_p[colA] = bits_out(p.out_f16, dv0[v] * (rs * cA) * sc, hit);
+          if (colB < ncols) orow_p[colB] = bits_out(p.out_f16, dv1[v] * (rs * cB) * sc, hit);
         }
       }
     }
   }
+  if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
 }
 
 // Q8: e4m3 operands (kind::f8f6f4, epilogue scales); a template parameter so
@@ -502,6 +515,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     // ---------------- epilogue (warps 2..5) ----------------
     const int sub = warp & 3;              // TMEM lane quarter this warp may access
     const int r = sub * 32 + lane;         // row within the tile
+    bool hit = false;                      // an fp16 output saturated
     int nb = 0;                            // same buffer sequence as the MMA issuer
     uint32_t ph_f = 0;                     // bit b: phase of acc_full[b]
     int slot = 0;
@@ -702,7 +716,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             }
             uint32_t pk[16];
 #pragma unroll
-            for (int v = 0; v < 16; ++v) pk[v] = pack_bf16(dv[2 * v] * scale, dv[2 * v + 1] * scale);
+            for (int v = 0; v < 16; ++v) pk[v] = pack_out(p.out_f16, dv[2 * v] * scale, dv[2 * v + 1] * scale, hit);
             stage_row32(box, lane, 4 * half, pk);
           }
           fence_proxy_async_smem();               // the box is read by the async proxy
@@ -731,10 +745,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             for (int v = 0; v < 4; ++v) {
               if (col0 + 8 * v < ncols) {
                 uint4 pk;
-                pk.x = pack_bf16(dv[8 * v + 0] * scale, dv[8 * v + 1] * scale);
-                pk.y = pack_bf16(dv[8 * v + 2] * scale, dv[8 * v + 3] * scale);
-                pk.z = pack_bf16(dv[8 * v + 4] * scale, dv[8 * v + 5] * scale);
-                pk.w = pack_bf16(dv[8 * v + 6] * scale, dv[8 * v + 7] * scale);
+                pk.x = pack_out(p.out_f16, dv[8 * v + 0] * scale, dv[8 * v + 1] * scale, hit);
+                pk.y = pack_out(p.out_f16, dv[8 * v + 2] * scale, dv[8 * v + 3] * scale, hit);
+                pk.z = pack_out(p.out_f16, dv[8 * v + 4] * scale, dv[8 * v + 5] * scale, hit);
+                pk.w = pack_out(p.out_f16, dv[8 * v + 6] * scale, dv[8 * v + 7] * scale, hit);
                 *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
               }
             }
@@ -746,6 +760,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     }
     // the staging boxes must not be released while a store still reads them
     if (EPI != EPI_ROUTER && kTmaStoreOut && lane == 0) bulk_wait_all();
+    if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
   }
 
   tc_fence_before();
@@ -1112,6 +1127,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
     // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
     const int sub = warp & 3;              // TMEM lane quarter this warp may access
     const int L = sub * 32 + lane;         // this thread's TMEM lane
+    bool hit = false;                      // an fp16 output saturated
     int nb = 0;
     uint32_t ph_f = 0;
     int slot = 0;
@@ -1167,7 +1183,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
               for (int v = 0; v < 32; ++v) {
                 if (c + v < w.tail) {
                   const float sc = (!w.sh && p.row_scale) ? __ldg(p.row_scale + trow0 + c + v) : 1.0f;
-                  outb[(trow0 + c + v) * ncols + col] = bf16_bits(dv[v] * sc);
+                  outb[(trow0 + c + v) * ncols + col] = bits_out(p.out_f16, dv[v] * sc, hit);
                 }
               }
             }
@@ -1223,10 +1239,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
               for (int v = 0; v < 4; ++v) {
                 if (col0 + 8 * v < ncols) {
                   uint4 pk;
-                  pk.x = pack_bf16(dv[8 * v + 0] * scale, dv[8 * v + 1] * scale);
-                  pk.y = pack_bf16(dv[8 * v + 2] * scale, dv[8 * v + 3] * scale);
-                  pk.z = pack_bf16(dv[8 * v + 4] * scale, dv[8 * v + 5] * scale);
-                  pk.w = pack_bf16(dv[8 * v + 6] * scale, dv[8 * v + 7] * scale);
+                  pk.x = pack_out(p.out_f16, dv[8 * v + 0] * scale, dv[8 * v + 1] * scale, hit);
+                  pk.y = pack_out(p.out_f16, dv[8 * v + 2] * scale, dv[8 * v + 3] * scale, hit);
+                  pk.z = pack_out(p.out_f16, dv[8 * v + 4] * scale, dv[8 * v + 5] * scale, hit);
+                  pk.w = pack_out(p.out_f16, dv[8 * v + 6] * scale, dv[8 * v + 7] * scale, hit);
                   *reinterpret_cast<uint4*>(out + col0 + 8 * v) = pk;
                 }
               }
@@ -1238,6 +1254,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(cluster_addr(&acc_empty[acc], 0));
     }
+    if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
   }
 
   // after a wait gave up, loads may still be landing in this CTA's shared
@@ -1503,6 +1520,7 @@ static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st)
     p.ncols_r = a.d; p.ncols_s = a.d;
     p.out_r = (uint16_t*)a.out_r; p.out_s = (uint16_t*)a.out_s;
     p.row_scale = a.row_scale;
+    p.out_f16 = a.out_f16;
   }
   if (!ok) return cudaErrorInvalidValue;
   p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
@@ -1605,6 +1623,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int which, cudaStream_t st) {
     p.ncols_r = a.d; p.ncols_s = a.d;
     p.out_r = (uint16_t*)a.out_r; p.out_s = (uint16_t*)a.out_s;
     p.row_scale = a.row_scale;
+    p.out_f16 = a.out_f16;
   }
   if (!ok) return cudaErrorInvalidValue;
   p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;

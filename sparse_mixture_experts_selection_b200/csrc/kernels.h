@@ -28,9 +28,12 @@ struct FfnArgs {
   float *as_r, *as_s;
   // training forward: U | V of every row ([rows, 2f] bf16) for the backward
   void *uv_r, *uv_s;
-  // 1: run both GEMMs on CTA pairs (tc_pair_rows()-row tiles, no merged
-  // tails; the group tables were built with that tile height)
+  // 1: run both GEMMs on CTA pairs (tc_pair_rows()-row tiles; the group
+  // tables were built with that tile height)
   int pair;
+  // 1: the down GEMM writes out_r / out_s in fp16 (saturating, MOE_DEVERR_RANGE)
+  // instead of bf16 -- the layer's internal slot and shared rows
+  int out_f16;
 };
 
 void launch_router_logits(const void* h, int dtype, const float* e, float* z, int T, int d, int E,
@@ -55,9 +58,10 @@ void launch_scatter(const int32_t* idx, const float* gates, const int* offsets,
 void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr, void* x_perm,
                    int d, int elem_bytes, int max_rows, int n_tok, int* err, cudaStream_t st,
                    const float* s_src = nullptr, float* s_dst = nullptr);
+// slot_f16: slot and shared rows are fp16 (a bf16 layer's internal rows)
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
                     void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
-                    int n_slot_rows, cudaStream_t st);
+                    int n_slot_rows, cudaStream_t st, int slot_f16 = 0);
 void launch_bias_update(const int* counts, float* b, float gamma, float* max_vio, int E, int K,
                         int T, cudaStream_t st);
 void launch_gather_map(const void* src, const int32_t* map, int64_t n_rows, int64_t n_src, int row_bytes,
@@ -132,6 +136,7 @@ struct BwdRouteArgs {
   const int32_t* sel_tok;    // sigmoid: every selected (t, j) by expert, tokens ascending
   const int* sel_off;        // [E + 1] its offsets
   int* err;
+  int slot_f16;              // slot rows in fp16 (the layer's), else bf16
 };
 void launch_bwd_route(const BwdRouteArgs& a, cudaStream_t st);        // dO, dL/dg
 void launch_zero_tail_rows(void* buf, const int* n_rows_ptr, int max_rows, int cols, cudaStream_t st);

@@ -607,9 +607,10 @@ __global__ void gather_map_kernel(const uint32_t* __restrict__ src, const int32_
 }
 
 // a8: y_t = res*h_t + sum_j shared[j,t] + sum_k slot[row_of[t,k]], fp32 in that order.
-template <typename T>
+// S: element type of the slot and shared rows (T, or fp16 for a bf16 layer's own).
+template <typename T, typename S = T>
 __global__ void __launch_bounds__(128)
-combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
+combine_kernel(const T* __restrict__ h, const S* __restrict__ slot, const S* __restrict__ shared,
                const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int K,
                int E_s, int add_residual, int n_slot_rows) {
   pdl_wait();
@@ -632,14 +633,14 @@ combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __r
     }
     for (int j = 0; j < E_s; ++j) {
       uint4 raw = *reinterpret_cast<const uint4*>(shared + ((size_t)j * n_tok + t) * d + c);
-      const T* v = reinterpret_cast<const T*>(&raw);
+      const S* v = reinterpret_cast<const S*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
     }
     for (int k = 0; k < K; ++k) {
       if (rows[k] < 0) continue;
       uint4 raw = *reinterpret_cast<const uint4*>(slot + (size_t)rows[k] * d + c);
-      const T* v = reinterpret_cast<const T*>(&raw);
+      const S* v = reinterpret_cast<const S*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
     }
@@ -658,9 +659,9 @@ combine_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __r
 // (registers capped at 80): more loads in flight per SM than the five the
 // unconstrained register count allows (measured 10-12 % faster), without the
 // spills that eight would cost.
-template <typename T, int KT>
+template <typename T, int KT, typename S = T>
 __global__ void __launch_bounds__(128, 6)
-combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* __restrict__ shared,
+combine_k_kernel(const T* __restrict__ h, const S* __restrict__ slot, const S* __restrict__ shared,
                  const int32_t* __restrict__ row_of, T* __restrict__ y, int n_tok, int d, int E_s,
                  int add_residual, int n_slot_rows) {
   pdl_wait();
@@ -688,14 +689,14 @@ combine_k_kernel(const T* __restrict__ h, const T* __restrict__ slot, const T* _
     }
     for (int j = 0; j < E_s; ++j) {
       const uint4 raw = __ldg(reinterpret_cast<const uint4*>(shared + ((size_t)j * n_tok + t) * d + c));
-      const T* v = reinterpret_cast<const T*>(&raw);
+      const S* v = reinterpret_cast<const S*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
     }
 #pragma unroll
     for (int k = 0; k < KT; ++k) {
       if (rows[k] < 0) continue;
-      const T* v = reinterpret_cast<const T*>(&sv[k]);
+      const S* v = reinterpret_cast<const S*>(&sv[k]);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(v[i]));
     }
@@ -988,14 +989,24 @@ void launch_gather(const void* h, const int32_t* perm_tok, const int* n_rows_ptr
 
 void launch_combine(const void* h, const void* slot, const void* shared, const int32_t* row_of,
                     void* y, int T, int d, int K, int E_s, int add_residual, int dtype,
-                    int n_slot_rows, cudaStream_t st) {
+                    int n_slot_rows, cudaStream_t st, int slot_f16) {
   // enough blocks to fill the GPU even for decode-sized batches
   const int nvec = d * (dtype == MOE_DTYPE_BF16 ? 2 : 4) / 16;
   int split = (2 * 148 + T - 1) / T;
   const int max_split = (nvec + 127) / 128;
   split = split < 1 ? 1 : (split > max_split ? max_split : split);
   const dim3 grid(T, split);
-  if (dtype == MOE_DTYPE_BF16 && (K == 2 || K == 4 || K == 6 || K == 8)) {
+  if (dtype == MOE_DTYPE_BF16 && slot_f16 && (K == 2 || K == 4 || K == 6 || K == 8)) {
+    const bf16* hh = (const bf16*)h;
+    const __half *sl = (const __half*)slot, *sh = (const __half*)shared;
+    bf16* yy = (bf16*)y;
+    auto kern = K == 8 ? combine_k_kernel<bf16, 8, __half> : K == 6 ? combine_k_kernel<bf16, 6, __half>
+              : K == 4 ? combine_k_kernel<bf16, 4, __half> : combine_k_kernel<bf16, 2, __half>;
+    launch_pdl(kern, grid, dim3(128), 0, st, hh, sl, sh, row_of, yy, T, d, E_s, add_residual, n_slot_rows);
+  } else if (dtype == MOE_DTYPE_BF16 && slot_f16) {
+    launch_pdl(combine_kernel<bf16, __half>, grid, dim3(128), 0, st, (const bf16*)h, (const __half*)slot,
+               (const __half*)shared, row_of, (bf16*)y, T, d, K, E_s, add_residual, n_slot_rows);
+  } else if (dtype == MOE_DTYPE_BF16 && (K == 2 || K == 4 || K == 6 || K == 8)) {
     const bf16 *hh = (const bf16*)h, *sl = (const bf16*)slot, *sh = (const bf16*)shared;
     bf16* yy = (bf16*)y;
     auto kern = K == 8 ? combine_k_kernel<bf16, 8> : K == 6 ? combine_k_kernel<bf16, 6>

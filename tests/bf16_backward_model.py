@@ -3,11 +3,11 @@ tolerance of the backward parity tests (test infrastructure, never the product
 path).
 
 The layer's GPU backward multiplies bf16 operands with fp32 accumulation and
-keeps these intermediates in bf16: the forward's U, V and A = SiLU(U) V and
-the gate-scaled expert output (slot); in the backward g*dy (dO), dU, dV, each
-expert's dX, the weight gradients and dh.  This model repeats the exact
-float64 arithmetic of the oracle's layer backward with a round to bf16 at
-exactly those points, and nowhere else.  Its distance from the oracle is the
+keeps these intermediates in bf16: the forward's U, V and A = SiLU(U) V; in
+the backward g*dy (dO), dU, dV, each expert's dX, the weight gradients and dh
+-- and the gate-scaled expert output (slot) in fp16.  This model repeats the
+exact float64 arithmetic of the oracle's layer backward with a round to bf16
+(fp16 for the slot) at exactly those points, and nowhere else.  Its distance from the oracle is the
 error those roundings alone cause; the parity bar must sit above it.
 """
 import numpy as np
@@ -20,12 +20,16 @@ def _rb(a):
     return mi.round_bf16(np.asarray(a, np.float32)).astype(np.float64)
 
 
+def _rh(a):
+    return np.asarray(a, np.float32).astype(np.float16).astype(np.float64)
+
+
 def _expert(x, wg, wu, wd, g, dy):
     x = np.asarray(x, np.float64)
     wg, wu, wd = (np.asarray(w, np.float64) for w in (wg, wu, wd))
     u, v = x @ wg.T, x @ wu.T
     a = _rb(u / (1.0 + np.exp(-u)) * v)
-    slot = _rb(g * (a @ wd.T))
+    slot = _rh(g * (a @ wd.T))
     ub, vb = _rb(u), _rb(v)
     sig = 1.0 / (1.0 + np.exp(-ub))
     do = _rb(g * dy)

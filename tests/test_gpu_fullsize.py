@@ -45,7 +45,7 @@ EXPECTED_KINDS = {
     "mixtral_8x14336": {"full", "full_with_tail", "merged_tail", "transposed"},
     "finegrained_64x1408": set(KINDS),
     "finegrained_64x1408_cf1.25": set(KINDS),
-    "deepseek_v3": {"full", "full_with_tail", "merged_tail", "padded"},
+    "deepseek_v3": set(KINDS),
     "deepseek_v3_decode": {"transposed"},
 }
 

@@ -45,6 +45,9 @@ SMALL = {
     "mixtral_pairs": W["mixtral_8x14336"].with_(T=2304, d_model=256, d_ffn=320),
     "finegrained_pairs": W["finegrained_64x1408"].with_(T=1100, d_model=192, E_r=8, E_s=2, K=4,
                                                         d_ffn=192, d_ffn_shared=136),
+    # T = 4 * 256 + 40: the shared experts' last 40 rows ride as merged tails
+    "finegrained_pairs_shared_tail": W["finegrained_64x1408"].with_(T=1064, d_model=192, E_r=8, E_s=2,
+                                                                    K=4, d_ffn=192, d_ffn_shared=136),
 }
 
 
@@ -350,7 +353,7 @@ def test_layer_gemm_tile_choice(name):
     w = SMALL[name]
     want = 32 if w.dtype == "f32" else (256 if w.T * w.K >= 512 * w.E_r else 128)
     assert moe.moe_expert_ffn_tile_rows(moe.config_for(w), w.E_r, w.T * w.K) == want
-    if name.endswith("_pairs"):
+    if "_pairs" in name:
         assert want == 256
 
 
@@ -394,6 +397,28 @@ def test_layer_independent(name):
         pytest.skip("a fragile token moved a capacity boundary")
     ok = same
     check_close(y[ok], ref["y"][ok], h[ok], tol_of(w), bool(w.add_residual), out_eps_of(w))
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "finegrained_pairs"])
+def test_layer_slot_saturation_reports_range(name):
+    """The layer keeps its slot and shared rows in fp16: down weights scaled by
+    2^20 (exact in bf16) push them past 65504; they saturate, the output stays
+    finite and the device error word reads MOE_DEVERR_RANGE -- on the
+    single-CTA and on the CTA-pair GEMMs.  The unscaled layer reports nothing."""
+    w = SMALL[name]
+    h, e, b = inputs(w)
+    HW = HostWeights(w)
+    Wd = HW.device()
+    L = Layer(w, Wd)
+    L.forward(to_dev(h, torch_dtype(w)), to_dev(e), to_dev(b))
+    assert L.device_error() == 0
+    Wd["down"].mul_(2.0 ** 20)
+    if Wd["sdown"] is not None:
+        Wd["sdown"].mul_(2.0 ** 20)
+    y = L.forward(to_dev(h, torch_dtype(w)), to_dev(e), to_dev(b))
+    assert L.device_error() == moe.DEVERR_RANGE
+    assert torch.isfinite(y.float()).all()
+    assert float(y.float().abs().max()) > 65504.0 / 2
 
 
 def test_layer_deterministic_and_workspace_reuse():
