@@ -296,6 +296,26 @@ def test_expert_ffn_pair_tiles():
     assert np.all(got[R:] == 7.0)                     # rows past offsets[n] untouched
 
 
+def test_expert_ffn_pair_tiles_all_empty():
+    """The CTA-pair GEMMs with no unit at all (every expert empty): the
+    launches end cleanly, no output row is touched, no error is set."""
+    n_exp, d, f = 4, 192, 200
+    cfg = moe.MoeConfig(T=64, d_model=d, E_r=n_exp, E_s=0, K=1, d_ffn=f, d_ffn_shared=0, score_fn=0,
+                        n_groups=1, topk_groups=1, group_topn=0, capacity_factor=0.0, dtype=1, add_residual=1)
+    max_rows = 512 * n_exp
+    assert moe.moe_expert_ffn_tile_rows(cfg, n_exp, max_rows) == 256
+    ws = moe.alloc_workspace(moe.moe_expert_ffn_workspace_size(cfg, n_exp, f, max_rows))
+    w = torch.zeros((n_exp, f, d), dtype=torch.bfloat16, device="cuda")
+    wd = torch.zeros((n_exp, d, f), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((max_rows, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((max_rows, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    offsets = torch.zeros(n_exp + 1, dtype=torch.int32, device="cuda")
+    moe.moe_expert_ffn(cfg, n_exp, f, max_rows, offsets, x, w, w, wd, None, out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    assert bool((out.float() == 7.0).all())
+
+
 @pytest.mark.parametrize("dtype,K", [("bf16", 3), ("f32", 3), ("bf16", 8), ("bf16", 2)])
 def test_combine_entry_fixed_order(dtype, K):
     T, d, E_s, R = 77, 64, 2, 200
