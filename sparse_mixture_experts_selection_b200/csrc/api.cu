@@ -25,8 +25,8 @@ constexpr int kChunkShift = 8;          // histogram chunk = 256 tokens (the sca
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
-// bytes of an activation element (h, y, x_perm, A, slots): bf16 for the bf16
-// and e4m3-weight layers, fp32 for fp32 layers
+// bytes of an activation element (h, y, x_perm, A, slots): 2 for the bf16 and
+// e4m3-weight layers (bf16; a layer's own slot rows fp16), 4 for fp32 layers
 size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_F32 ? 4 : 2; }
 int act_dtype(int dtype) { return dtype == MOE_DTYPE_F32 ? MOE_DTYPE_F32 : MOE_DTYPE_BF16; }
 bool is_q8(int dtype) { return dtype == MOE_DTYPE_BF16_E4M3; }
