@@ -91,12 +91,11 @@ void launch_ffn_simt(const FfnArgs& a, int which, cudaStream_t st);
 // ks split-K ranges (summed in order by the select kernel).
 // At most kRouterMaxSplits partials (kRouterMaxSplitsSmallT for batches of
 // at most kRouterSmallT tokens, where one row tile leaves most SMs idle unless
-// the reduction is cut finer); the select kernel adds them kRouterPartChunk
-// at a time.
+// the reduction is cut finer); the select kernel adds them in split order,
+// loading 64 partial values per lane at a time.
 constexpr int kRouterMaxSplits = 16;
 constexpr int kRouterMaxSplitsSmallT = 64;
 constexpr int kRouterSmallT = 1024;
-constexpr int kRouterPartChunk = 16;
 constexpr int kRouterMaxKbPerSplit = 24;
 inline int router_max_splits(int T) { return T <= kRouterSmallT ? kRouterMaxSplitsSmallT : kRouterMaxSplits; }
 void router_split_plan(int T, int d, int E, int n_sms, int* ks, int* per);

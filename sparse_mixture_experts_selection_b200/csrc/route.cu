@@ -97,25 +97,33 @@ select_kernel(const float* __restrict__ in, int n_parts, int in_is_scores, const
   const float* row = in + (size_t)t * E;
 
   float s[KPL], key[KPL];
+  // logits from split-K partial sums, added in split order (deterministic):
+  // each round loads PC partials of all KPL experts of this lane at once
+  // (KPL * PC = 64 loads in flight), so a token with many partials -- small
+  // batches are split finest -- waits for n_parts / PC load latencies, not
+  // for KPL * n_parts / PC of them
+  constexpr int PC = 64 / KPL > 0 ? 64 / KPL : 1;
 #pragma unroll
-  for (int j = 0; j < KPL; ++j) {
-    int ex = j * kWarp + lane;
-    // logits from split-K partial sums: the partials are loaded
-    // kRouterPartChunk at a time (all loads of a chunk in flight together)
-    // and added in split order (deterministic)
-    float acc = 0.f;
-    for (int q0 = 0; q0 < n_parts; q0 += kRouterPartChunk) {
-      float part[kRouterPartChunk];
+  for (int j = 0; j < KPL; ++j) s[j] = 0.f;
+  for (int q0 = 0; q0 < n_parts; q0 += PC) {
+    float part[KPL][PC];
 #pragma unroll
-      for (int q = 0; q < kRouterPartChunk; ++q)
-        part[q] = (q0 + q < n_parts && ex < E) ? row[(size_t)(q0 + q) * T * E + ex] : 0.f;
-      acc = q0 == 0 ? part[0] : __fadd_rn(acc, part[0]);
+    for (int j = 0; j < KPL; ++j) {
+      const int ex = j * kWarp + lane;
 #pragma unroll
-      for (int q = 1; q < kRouterPartChunk; ++q)
-        if (q0 + q < n_parts) acc = __fadd_rn(acc, part[q]);
+      for (int q = 0; q < PC; ++q)
+        part[j][q] = (q0 + q < n_parts && ex < E) ? row[(size_t)(q0 + q) * T * E + ex] : 0.f;
     }
-    s[j] = ex < E ? acc : 0.f;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+#pragma unroll
+      for (int q = 0; q < PC; ++q)
+        if (q0 + q < n_parts) s[j] = (q0 + q == 0) ? part[j][q] : __fadd_rn(s[j], part[j][q]);
+    }
   }
+#pragma unroll
+  for (int j = 0; j < KPL; ++j)
+    if (j * kWarp + lane >= E) s[j] = 0.f;
   if (!in_is_scores) {
     if (z_out) {
 #pragma unroll
