@@ -101,6 +101,7 @@ struct Params {
   // EPI_ROUTER: z partial sums over split-K ranges of the virtual reduction
   // [h | h | h] . [e_hi | e_mid | e_lo]^T (no group table)
   int r_T, r_E, r_mtiles, r_ntiles, r_ks, r_nkd, r_per;
+  int r_n;                    // MMA N of the router: round16(E) up to 256 (fewer experts: a narrower tile)
   float* zpart;               // [r_ks, r_T, r_E]
   // dynamic schedule: units are claimed from this zeroed counter (null: static
   // round-robin over the CTAs)
@@ -400,7 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         // that hold its N rows
         const int n_sub = w.n16 ? (w.n16 + A_SUB_ROWS - 1) / A_SUB_ROWS : 0;
         const int t_sub = (w.t16 + A_SUB_ROWS - 1) / A_SUB_ROWS;
-        const uint32_t tx = (uint32_t)((n_sub ? n_sub * A_SUB_BYTES : A_BYTES) + t_sub * A_SUB_BYTES + B_BYTES);
+        const uint32_t b_bytes = EPI == EPI_ROUTER ? (uint32_t)p.r_n * BK * 2 : (uint32_t)B_BYTES;
+        const uint32_t tx = (uint32_t)((n_sub ? n_sub * A_SUB_BYTES : A_BYTES) + t_sub * A_SUB_BYTES) + b_bytes;
         for (int i = 0; i < w.nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) goto producer_done;
           const TileCoords<EPI> c = tile_coords<EPI>(p, w, i);
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         // the two 128-row halves of W_down's 256) against the N = n16 rows,
         // into accumulator columns [0, n16) and [128, 128 + n16)
         constexpr bool q8 = EPI != EPI_ROUTER && Q8;
-        const uint32_t idesc_n = q8 ? IDESC_Q8 : IDESC;
+        const uint32_t idesc_n = q8 ? IDESC_Q8 : EPI == EPI_ROUTER ? idesc_bf16_f32(BM, p.r_n) : IDESC;
         const uint32_t idesc_t = q8 ? idesc_e4m3_f32(BM, w.n16 ? w.n16 : 16) : idesc_bf16_f32(BM, w.n16 ? w.n16 : 16);
         const uint32_t idesc_tail = q8 ? idesc_e4m3_f32(BM, w.t16 ? w.t16 : 16) : idesc_bf16_f32(BM, w.t16 ? w.t16 : 16);
         // a unit with a merged tail holds buffer 0 (full tile) and buffer 1 (tail)
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         const int ks = nt % p.r_ks, ct = nt / p.r_ks;
         float* zrow = p.zpart + ((size_t)ks * p.r_T + m) * p.r_E;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < p.r_n; c += 32) {
           float dv[32];
           tmem_ld32(tb + c, dv);
           const int col0 = ct * BN + c;
@@ -1393,12 +1395,15 @@ cudaError_t launch_router_tc(const void* h, const float* e, void* e3, float* zpa
   bool ok = true;
   ok &= make_tmap(&p.a_r, h, (uint64_t)T, d, BM);
   ok &= make_tmap(&p.a_s, h, (uint64_t)T, d, BM);
-  ok &= make_tmap(&p.b0_r, e3, (uint64_t)3 * E, d, BN);
-  ok &= make_tmap(&p.b1_r, e3, (uint64_t)3 * E, d, BN);
-  ok &= make_tmap(&p.b0_s, e3, (uint64_t)3 * E, d, BN);
-  ok &= make_tmap(&p.b1_s, e3, (uint64_t)3 * E, d, BN);
+  // fewer than 256 experts: an N = round16(E) tile (the box then holds only
+  // this part's centroid rows, not the next part's)
+  const int rn = E >= BN ? BN : ((E + 15) / 16) * 16;
+  ok &= make_tmap(&p.b0_r, e3, (uint64_t)3 * E, d, rn);
+  ok &= make_tmap(&p.b1_r, e3, (uint64_t)3 * E, d, rn);
+  ok &= make_tmap(&p.b0_s, e3, (uint64_t)3 * E, d, rn);
+  ok &= make_tmap(&p.b1_s, e3, (uint64_t)3 * E, d, rn);
   if (!ok) return cudaErrorInvalidValue;
-  p.r_T = T; p.r_E = E;
+  p.r_T = T; p.r_E = E; p.r_n = rn;
   p.r_mtiles = (T + BM - 1) / BM;
   p.r_ntiles = (E + BN - 1) / BN;
   p.r_ks = ks; p.r_per = per;
