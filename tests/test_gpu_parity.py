@@ -187,6 +187,40 @@ def test_permute_bit_exact(cf):
     assert np.array_equal(dev["x_perm"].cpu().numpy()[:n], h[ref.perm_tok])
 
 
+@pytest.mark.parametrize("dtype,d", [("f32", 8192), ("bf16", 4104), ("f32", 8)])
+def test_permute_row_gather_widths(dtype, d):
+    """x_perm = h[perm_tok] bit for bit across row widths: 32 KB fp32 rows leave
+    room for only three row buffers in the bulk-copy ring, so the row gather
+    falls back to its per-lane copy; 8208-byte bf16 rows take the ring with
+    an odd number of 16-byte chunks; 32-byte rows the ring's smallest rows;
+    rows past the kept ones stay untouched."""
+    T, E, K = 300, 16, 3
+    rng = np.random.default_rng(11)
+    s = mo.sigmoid_scores(rng.normal(size=(T, E)).astype(np.float32))
+    idx = mo.select_experts(s, np.zeros(E, np.float32), K)
+    h = rng.normal(size=(T, d)).astype(np.float32)
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    if dtype == "bf16":
+        h = mi.round_bf16(h)
+    cfg = moe.MoeConfig(T=T, d_model=d, E_r=E, E_s=0, K=K, d_ffn=64, d_ffn_shared=0, score_fn=0,
+                        n_groups=1, topk_groups=1, group_topn=0, capacity_factor=1.0,
+                        dtype=0 if dtype == "f32" else 1, add_residual=1)
+    ws = moe.alloc_workspace(moe.moe_workspace_size(cfg))
+    z = lambda *sh: torch.empty(sh, dtype=torch.int32, device="cuda")
+    x_perm = torch.full((T * K, d), 3.0, dtype=dt, device="cuda")
+    offsets, perm_tok = z(E + 1), z(T * K)
+    moe.moe_permute(cfg, to_dev(idx.astype(np.int32), torch.int32), None, to_dev(h, dt), offsets, perm_tok,
+                    z(T, K), z(E), None, x_perm, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    ref = mo.dispatch(idx, E, 1.0)
+    n = int(ref.offsets[-1])
+    assert n < T * K                                  # capacity 1.0 drops some pairs
+    got = x_perm.float().cpu().numpy()
+    assert np.array_equal(got[:n], h[ref.perm_tok])
+    assert np.all(got[n:] == 3.0)
+
+
 def test_permute_rejects_bad_expert_index():
     """An out-of-range expert index sets the device error word (no fault)."""
     T, E, K = 64, 8, 2
