@@ -819,11 +819,18 @@ constexpr int P_M = 2 * BM;                     // 256 rows per pair tile
 constexpr int P_B_BYTES = (BN / 2) * BK * 2;    // 16 KB: this CTA's half of the weight tile
 constexpr int P_T_BYTES = A_SUB_BYTES;          // 4 KB: a 32-row box of this CTA's tail rows
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES + P_T_BYTES;
-constexpr int P_STAGES = 6;
 constexpr int P_XCHG_BYTES = 32 * 64 * 4;       // 8 KB: up values of 32 tail rows x 64 columns
-constexpr size_t P_SMEM = (size_t)P_STAGES * P_STAGE_BYTES + P_XCHG_BYTES + 1024 + CTRL_BYTES;
+// Down GEMMs with short units (at most kTmaOutMaxKb k-blocks) stage their
+// outputs in shared memory for TMA stores, as the single-CTA down GEMM does:
+// the 32 KB of boxes cost one of the six stages.
+template <bool TMA_OUT> constexpr int p_stages() { return TMA_OUT ? 5 : 6; }
+template <bool TMA_OUT> constexpr int p_extra_bytes() { return TMA_OUT ? 4 * 2 * OUT_BOX_BYTES : P_XCHG_BYTES; }
+template <bool TMA_OUT> constexpr size_t p_smem() {
+  return (size_t)p_stages<TMA_OUT>() * P_STAGE_BYTES + p_extra_bytes<TMA_OUT>() + 1024 + CTRL_BYTES;
+}
+constexpr size_t P_SMEM = p_smem<false>();
 constexpr uint32_t P_IDESC = idesc_bf16_f32(P_M, BN);
-static_assert(P_SMEM <= 232448, "shared memory per CTA");
+static_assert(p_smem<false>() <= 232448 && p_smem<true>() <= 232448, "shared memory per CTA");
 static_assert(kPairMergeMax <= 2 * A_SUB_ROWS, "a tail's half fits one 32-row box");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -951,15 +958,18 @@ __device__ __forceinline__ bool pair_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
-template <int EPI>
+template <int EPI, bool TMA_OUT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  constexpr int P_STAGES = p_stages<TMA_OUT>();
+  constexpr bool kTmaStoreOut = TMA_OUT && EPI == EPI_SCALE;
   uint8_t* sA = smem;
   uint8_t* sB = smem + P_STAGES * A_BYTES;
   uint8_t* sT = sB + P_STAGES * P_B_BYTES;
-  float* xchg = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES + P_XCHG_BYTES);
+  float* xchg = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES);       // gate/up tails
+  uint8_t* sOut = smem + P_STAGES * P_STAGE_BYTES;                               // staging boxes (TMA_OUT)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES + p_extra_bytes<TMA_OUT>());
   uint64_t* empty = full + P_STAGES;
   uint64_t* acc_full = empty + P_STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -985,6 +995,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
   if (warp == 1 && lane == 0) {
     prefetch_tmap(&p.a_r); prefetch_tmap(&p.a_s); prefetch_tmap(&p.a32_r); prefetch_tmap(&p.a32_s);
     prefetch_tmap(&p.b0_r); prefetch_tmap(&p.b1_r); prefetch_tmap(&p.b0_s); prefetch_tmap(&p.b1_s);
+    if (kTmaStoreOut) { prefetch_tmap(&p.o_r); prefetch_tmap(&p.o_s); }
   }
   __syncthreads();
   cluster_sync_all();          // both CTAs' barriers are initialised before either signals the other
@@ -1130,6 +1141,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
     const int sub = warp & 3;              // TMEM lane quarter this warp may access
     const int L = sub * 32 + lane;         // this thread's TMEM lane
     bool hit = false;                      // an fp16 output saturated
+    uint8_t* my_boxes = sOut + sub * 2 * OUT_BOX_BYTES;   // this warp's two staging boxes (TMA_OUT)
+    int n_boxes = 0;
     int nb = 0;
     uint32_t ph_f = 0;
     int slot = 0;
@@ -1229,6 +1242,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
               }
             }
           }
+        } else if (kTmaStoreOut && m0 + 32 <= w.rows) {
+          // every row of this warp is valid: 64 columns at a time through a
+          // staging box and one TMA store (whole 128-byte lines)
+          const float scale = (!w.sh && p.row_scale) ? __ldg(p.row_scale + orow) : 1.0f;
+          const CUtensorMap* om = w.sh ? &p.o_s : &p.o_r;
+          const int orow0 = (int)(orow - (size_t)lane);
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 64) {
+            uint8_t* box = my_boxes + (n_boxes & 1) * OUT_BOX_BYTES;
+            if (lane == 0) bulk_wait_read_1();    // the store that last read this box is done reading
+            __syncwarp();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              float dv[32];
+              tmem_ld32(tb + c + 32 * half, dv);
+              uint32_t pk[16];
+#pragma unroll
+              for (int v = 0; v < 16; ++v) pk[v] = pack_out(p.out_f16, dv[2 * v] * scale, dv[2 * v + 1] * scale, hit);
+              stage_row32(box, lane, 4 * half, pk);
+            }
+            fence_proxy_async_smem();             // the box is read by the async proxy
+            __syncwarp();
+            if (lane == 0) {
+              const int x = w.nt * BN + c;
+              if (x < ncols) tma_store_2d(om, box, x, orow0);   // columns past ncols are clipped
+              bulk_commit();                      // one group per box, even an empty one
+            }
+            ++n_boxes;
+          }
         } else {
           const float scale = (!w.sh && p.row_scale && valid) ? __ldg(p.row_scale + orow) : 1.0f;
 #pragma unroll 1
@@ -1256,6 +1298,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) pair_gemm_kernel(const __grid_
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(cluster_addr(&acc_empty[acc], 0));
     }
+    // the staging boxes must not be released while a store still reads them
+    if (kTmaStoreOut && lane == 0) bulk_wait_all();
     if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
   }
 
@@ -1460,6 +1504,8 @@ static void pair_attributes() {
   if (dev < 64 && !attr_done[dev]) {
     cudaFuncSetAttribute(pair_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
     cudaFuncSetAttribute(pair_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    cudaFuncSetAttribute(pair_gemm_kernel<EPI_SCALE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)p_smem<true>());
     attr_done[dev] = true;
   }
 }
@@ -1526,14 +1572,21 @@ static cudaError_t launch_ffn_pair(const FfnArgs& a, int which, cudaStream_t st)
     p.out_r = (uint16_t*)a.out_r; p.out_s = (uint16_t*)a.out_s;
     p.row_scale = a.row_scale;
     p.out_f16 = a.out_f16;
+    ok &= make_tmap(&p.o_r, a.out_r, (uint64_t)a.max_rows_r, a.d, OUT_BOX_ROWS);
+    ok &= make_tmap(&p.o_s, has_s ? a.out_s : a.out_r, rows_s, a.d, OUT_BOX_ROWS);
   }
   if (!ok) return cudaErrorInvalidValue;
   p.tile_counter = a.tile_counters ? a.tile_counters + which : nullptr;
-  auto kern = which == 0 ? pair_gemm_kernel<EPI_SWIGLU> : pair_gemm_kernel<EPI_SCALE>;
+  // down GEMM with short units: outputs through the staging boxes and TMA stores
+  const int kb_r = (a.f_r + p.bk - 1) / p.bk, kb_s = (p.k_s + p.bk - 1) / p.bk;
+  const bool tma_out = which == 1 && std::max(kb_r, has_s ? kb_s : 0) <= kTmaOutMaxKb;
+  auto kern = which == 0 ? pair_gemm_kernel<EPI_SWIGLU>
+            : tma_out ? pair_gemm_kernel<EPI_SCALE, true> : pair_gemm_kernel<EPI_SCALE>;
+  const size_t smem = tma_out ? p_smem<true>() : P_SMEM;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pair_grid((const void*)kern, P_SMEM));
+  cfg.gridDim = dim3(pair_grid((const void*)kern, smem));
   cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = P_SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
