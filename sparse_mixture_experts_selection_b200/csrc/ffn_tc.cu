@@ -211,6 +211,8 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tmap, const void
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // all but the most recent bulk group of this thread have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every bulk group of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Write 16 bf16 pairs (32 columns) of this lane's row into the staging box:
@@ -322,6 +324,76 @@ __device__ __noinline__ void epilogue_transposed(const Params& p, bool sh, uint1
         }
       }
     }
+  }
+  if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
+}
+
+// The same for a down GEMM (EPI_SCALE) whose warps own staging boxes: 32 rows
+// at a time, the warp writes its 32 columns x 32 rows of each half (lane =
+// column) into a padded shared tile and reads them back by rows (lane = row),
+// so every output row leaves as 16-byte vectors instead of one 2-byte store
+// per value, and each row's gate is loaded once (lane = row) and broadcast.
+// tile: two 32 x kTrLine halves (80-byte lines: no bank conflicts either way).
+constexpr int kTrLine = 40;
+static_assert(2 * 32 * kTrLine * 2 <= 2 * OUT_BOX_BYTES, "the tile fits a warp's two staging boxes");
+__device__ __noinline__ void epilogue_transposed_staged(const Params& p, bool sh, uint16_t* out0, size_t row0,
+                                                        int rv, int n16, int colA, int ncols, uint32_t tb,
+                                                        const float* xs, const float* wsA, uint16_t* tile,
+                                                        int lane) {
+  const int colB = colA + BN / 2;
+  float cA = 1.0f, cB = 1.0f;
+  if (xs && colA < ncols) cA = __ldg(wsA + colA);
+  if (xs && colB < ncols) cB = __ldg(wsA + colB);
+  const int colA0 = colA - lane, colB0 = colB - lane;     // the warp's first column of each half
+  uint16_t* tA = tile;
+  uint16_t* tB = tile + 32 * kTrLine;
+  bool hit = false;
+#pragma unroll 1
+  for (int c = 0; c < n16; c += 32) {
+    float dv0[32], dv1[32];
+    tmem_ld32(tb + c, dv0);
+    tmem_ld32(tb + BN / 2 + c, dv1);
+    const int tl = c + lane;                               // the row this lane loads for and stores
+    float rs_l = 1.0f, sc_l = 1.0f;
+    if (tl < rv) {
+      if (xs) rs_l = __ldg(xs + tl);
+      if (!sh && p.row_scale) sc_l = __ldg(p.row_scale + row0 + tl);
+    }
+    bool hA = false, hB = false;
+#pragma unroll
+    for (int v = 0; v < 32; ++v) {
+      const float rs = xs ? __shfl_sync(0xffffffffu, rs_l, v) : 1.0f;
+      const float sc = __shfl_sync(0xffffffffu, sc_l, v);
+      uint16_t a = 0, b = 0;
+      if (c + v < rv) {
+        a = bits_out(p.out_f16, dv0[v] * (rs * cA) * sc, hA);
+        b = bits_out(p.out_f16, dv1[v] * (rs * cB) * sc, hB);
+      }
+      tA[v * kTrLine + lane] = a;
+      tB[v * kTrLine + lane] = b;
+    }
+    hit |= (hA && colA < ncols) || (hB && colB < ncols);
+    __syncwarp();
+    if (tl < rv) {
+      uint16_t* orow = out0 + (size_t)tl * ncols;
+      const uint16_t* sa = tA + lane * kTrLine;
+      const uint16_t* sb = tB + lane * kTrLine;
+      if (colA0 + 32 <= ncols) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(orow + colA0 + 8 * q) = *reinterpret_cast<const uint4*>(sa + 8 * q);
+      } else {
+        for (int j = 0; j < 32 && colA0 + j < ncols; ++j) orow[colA0 + j] = sa[j];
+      }
+      if (colB0 + 32 <= ncols) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(orow + colB0 + 8 * q) = *reinterpret_cast<const uint4*>(sb + 8 * q);
+      } else {
+        for (int j = 0; j < 32 && colB0 + j < ncols; ++j) orow[colB0 + j] = sb[j];
+      }
+    }
+    __syncwarp();                                          // the tile is rewritten by the next 32 rows
   }
   if (hit) set_device_error(p.err, MOE_DEVERR_RANGE);
 }
@@ -569,16 +641,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         if (!mbar_wait(&acc_full[1], (ph_f >> 1) & 1u, abort_flag, p.err)) break;
         ph_f ^= 2u;
         tc_fence_after();
-        epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
-                                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
-                                 xs ? xs + BM : nullptr, wsA, wsB, uv0 ? uv0 + (size_t)BM * 2 * ncols : nullptr);
+        if (EPI == EPI_SCALE && kTmaStoreOut) {
+          if (lane == 0) bulk_wait_read_0();      // no store still reads this warp's boxes
+          __syncwarp();
+          epilogue_transposed_staged(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
+                                     tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
+                                     xs ? xs + BM : nullptr, wsA, reinterpret_cast<uint16_t*>(my_boxes), lane);
+        } else {
+          epilogue_transposed<EPI>(p, sh, out0 + (size_t)BM * ncols, row0 + BM, w.tail, w.t16, colA, ncols,
+                                   tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)BN,
+                                   xs ? xs + BM : nullptr, wsA, wsB, uv0 ? uv0 + (size_t)BM * 2 * ncols : nullptr);
+        }
         tc_fence_before();
         mbar_arrive(&acc_empty[1]);
       }
       if (!mbar_wait(&acc_full[acc], (ph_f >> acc) & 1u, abort_flag, p.err)) break;
       ph_f ^= 1u << acc;
       tc_fence_after();
-      if (EPI != EPI_ROUTER && w.n16) {
+      if (EPI == EPI_SCALE && kTmaStoreOut && w.n16) {
+        if (lane == 0) bulk_wait_read_0();        // no store still reads this warp's boxes
+        __syncwarp();
+        epilogue_transposed_staged(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb,
+                                   xs, wsA, reinterpret_cast<uint16_t*>(my_boxes), lane);
+      } else if (EPI != EPI_ROUTER && w.n16) {
         epilogue_transposed<EPI>(p, sh, out0, row0, min(BM, rows - mt * BM), w.n16, colA, ncols, tb,
                                  xs, wsA, wsB, uv0);
       } else if (EPI == EPI_ROUTER) {
