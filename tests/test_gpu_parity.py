@@ -243,9 +243,12 @@ def test_permute_rejects_bad_expert_index():
 # experts (a6-a7), combine (a8), bias (a9)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_expert_ffn_entry(dtype):
-    n_exp, d, f = 5, 192, 200
+@pytest.mark.parametrize("dtype,d", [("bf16", 192), ("bf16", 200), ("f32", 192)])
+def test_expert_ffn_entry(dtype, d):
+    """Rows 130 and 257 end in merged tails, the 1-row expert is a transposed
+    tile; d = 200 leaves the down GEMM's last 32-column block of a warp
+    partly past the output width (the staged epilogue's element-wise edge)."""
+    n_exp, f = 5, 200
     rows = np.array([0, 130, 0, 257, 1], dtype=np.int64)     # empty groups and ragged tiles
     offsets = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
     R = int(offsets[-1])
